@@ -1,0 +1,539 @@
+#!/usr/bin/env python
+"""Throughput of the attention-prologue kernels on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one rope_split_store_paged_ragged call (RoPE of Q and K, split, paged K/V store)
+over the Llama-3-8B-shaped ragged prefill batch: 32 Q / 8 KV heads, head_dim 128, 8
+sequences with seeded lengths U[256, 2048], page_size 128, half-split RoPE, bf16.  Inputs are
+resident in HBM; a 256 MiB memset flushes L2 before every step, outside the timed events.
+`value` = tokens processed by all ranks / the max over ranks of the summed per-step device
+time (CUDA events on the launching stream).  Under torchrun every rank runs its own replica
+of the workload (its own seeded batch: weak scaling, no collective on the data path).
+
+Also printed (same JSON line): `e2e` (the same step through the Python binding with the
+inputs copied from pinned host memory and q_out copied back inside the timed region),
+`roofline` (algorithmic bytes of one launch / mean launch time, against the measured HBM
+copy bandwidth), `cpu_baseline` (the CPU oracle on the host cores), `clocks` (nvidia-smi
+samples during the timed region), and `entry_points` (the other four entry points on their
+named workloads, at N=1).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused RoPE+KV-store tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/rope_store.cu",
+                  "rope_paged_kv_b200/csrc/device_utils.cuh"]
+PROFILE = "profiles/rope_split_store_paged_ragged_llama3_8b_prefill.md"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other entry points and the CPU baseline")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ small utilities --
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs: torch copy_ of 1 Gi bf16)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
+
+
+def profiled_traffic():
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel sources (else None)."""
+    p = os.path.join(ROOT, PROFILE)
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons, with host timestamps."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str, interval_ms: int = 50):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", gpu_id, "-lms", str(interval_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[1]), float(parts[2]),
+                                     [n for n, v in zip(self.NAMES, parts[5:9])
+                                      if v.lower() == "active"]))
+            except ValueError:
+                pass
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside or self.samples
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({r for s in use for r in s[3]})
+        return {"sm_mhz": statistics.median(s[1] for s in use),
+                "sm_max_mhz": max(s[2] for s in use), "reasons": reasons,
+                "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# ------------------------------------------------------------- algorithmic bytes --
+
+def freqs_bytes(w_rope, positions) -> int:
+    return len(set(positions)) * w_rope.rope_dim * w_rope.table.element_size()
+
+
+def positions_ragged(lengths, cache_lengths):
+    pos = []
+    for n, c in zip(lengths, cache_lengths):
+        pos.extend(range(int(c), int(c) + n))
+    return pos
+
+
+def bytes_ragged(w) -> int:
+    """QKV rows read + Q rows written + K and V rows stored + distinct freqs_cis rows."""
+    D, Hq, Hk = w.cache.head_dim, w.n_q_heads, w.cache.n_kv_heads
+    eb = w.qkv.element_size()
+    row = (Hq + 2 * Hk) * D * eb
+    return w.total_tokens * 2 * row + freqs_bytes(
+        w.rope, positions_ragged(w.lengths, w.cache.cache_lengths.tolist()))
+
+
+def bytes_dual(w) -> int:
+    D, eb = w.main_cache.head_dim, w.input.element_size()
+    heads = (w.main_q_heads + 2 * w.main_cache.n_kv_heads + w.index_q_heads +
+             w.index_cache.n_kv_heads)
+    return w.total_tokens * 2 * heads * D * eb + freqs_bytes(
+        w.rope, positions_ragged(w.lengths, w.main_cache.cache_lengths.tolist()))
+
+
+def bytes_radd(w) -> int:
+    """a read + cache rows read + cache rows written."""
+    return w.a.shape[0] * 3 * w.a.shape[1] * w.a.element_size()
+
+
+def bytes_bshd(w) -> int:
+    """Q read + output written; K rows read + written in place (valid tokens); freqs rows."""
+    B, S, Hq, D = w.q_proj.shape
+    eb = w.q_proj.element_size()
+    valid = [min(int(v), S) for v in w.valid_lengths.tolist()]
+    k_rows = sum(valid) * w.cache.n_kv_heads * D * eb * 2
+    pos = [int(c) + s for c, v in zip(w.cache.cache_lengths.tolist(), valid) for s in range(v)]
+    return B * S * Hq * D * eb * 2 + k_rows + freqs_bytes(w.rope, pos)
+
+
+# ----------------------------------------------------------------------- our arm --
+
+def run_ours(args):
+    import ctypes
+
+    import torch
+    import torch.distributed as dist
+
+    import rope_paged_kv_b200 as rs
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def d(t):
+        return t.to(dev)
+
+    # this rank's replica: its own seeded batch
+    w = W.llama3_8b_prefill(seed=1000 * rank)
+    kv = w.cache
+    storage = d(kv.storage)
+    cache = rs.PagedCache(storage[kv.k_offset:], storage[kv.v_offset:], d(kv.page_table),
+                          d(kv.cache_lengths), kv.n_kv_heads, kv.head_dim, kv.page_size,
+                          kv.num_pages, kv.num_layers, kv.page_stride, kv.layer_stride,
+                          kv.slot_stride, kv.head_stride)
+    qkv, offs, q_out = d(w.qkv), d(w.offsets), d(w.q_out)
+    freqs = rs.Freqs(d(w.rope.table), w.rope.interleaved)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # the C entry point with its arguments marshalled once
+    lib = rs.raw_library()
+    c_f, c_kv = freqs.c(), cache.c()
+    c_args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
+              offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), w.layer_idx,
+              q_out.data_ptr(), q_out.stride(0), err.data_ptr(), stream.cuda_stream)
+
+    def step():
+        st = lib.rope_split_store_paged_ragged(*c_args)
+        if st != 0:
+            raise rs.RopeError(st, "rope_split_store_paged_ragged")
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, "device error bits set on the benchmark workload"
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for k in range(K):
+        flush.zero_()
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    dev_ms = sum(a.elapsed_time(b) for a, b in ev)
+    launches = K
+
+    # end to end: pinned host inputs in, q_out back out, through the Python binding
+    qkv_h = w.qkv.pin_memory()
+    offs_h, cl_h, pt_h = (w.offsets.pin_memory(), kv.cache_lengths.pin_memory(),
+                          kv.page_table.pin_memory())
+    q_out_h = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (qkv_h, offs_h, cl_h, pt_h))
+    d2h = q_out_h.numel() * q_out_h.element_size()
+    K_e2e = max(1, min(K, 200))
+
+    def e2e_step():
+        qkv.copy_(qkv_h, non_blocking=True)
+        offs.copy_(offs_h, non_blocking=True)
+        cache.cache_lengths.copy_(cl_h, non_blocking=True)
+        cache.page_table.copy_(pt_h, non_blocking=True)
+        rs.rope_split_store_paged_ragged(qkv, w.n_q_heads, offs, freqs, cache, w.layer_idx,
+                                         q_out, err)
+        q_out_h.copy_(q_out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K_e2e)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(K_e2e):
+        flush.zero_()
+        ev2[k][0].record(stream)
+        e2e_step()
+        ev2[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    sampler.stop()
+
+    tokens = torch.tensor([float(w.total_tokens)], device=dev, dtype=torch.float64)
+    times = torch.tensor([dev_ms, e2e_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(tokens, op=dist.ReduceOp.SUM)
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    tok_all = float(tokens.item())
+    dev_ms_max, e2e_ms_max = (float(x) for x in times.tolist())
+
+    extras = {}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        extras = run_entry_points(rs, W, dev, flush)
+        extras["rope_split_store_paged_ragged"] = {
+            "workload": w.name, "tokens": w.total_tokens,
+            "us_per_launch": round(dev_ms / K * 1e3, 2),
+            "tokens_per_s": round(w.total_tokens * K / (dev_ms / 1e3), 1),
+            "algorithmic_gbs": round(bytes_ragged(w) * K / (dev_ms / 1e3) / 1e9, 1)}
+        cpu = cpu_baseline(W)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_src = measured_peak()
+    alg = bytes_ragged(w)
+    mean_s = dev_ms / K / 1e3
+    achieved = alg / mean_s / 1e9
+    for v in extras.values():
+        if "algorithmic_gbs" in v:
+            v["frac_of_measured_hbm"] = round(v["algorithmic_gbs"] / peak, 3)
+    line = {
+        "metric": METRIC, "value": round(tok_all * K / (dev_ms_max / 1e3), 1), "unit": UNIT,
+        "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": round(dev_ms_max / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of a Llama-3-8B ragged prefill)",
+        "config": {"workload": w.name, "entry_point": "rope_split_store_paged_ragged",
+                   "tokens_per_rank": w.total_tokens, "batch": len(w.lengths),
+                   "lengths": w.lengths, "n_q_heads": w.n_q_heads,
+                   "n_kv_heads": kv.n_kv_heads, "head_dim": kv.head_dim,
+                   "page_size": kv.page_size, "rope": "half-split, rope_dim 128, theta 5e5, "
+                   "freqs_cis f32 [8192, 128]", "cache_dtype": "bf16",
+                   "l2": "flushed before every step (256 MiB memset outside the timed events)",
+                   "parallelism": f"replicas x{world} (each rank its own batch, no collective)"},
+        "gpu_launches": launches,
+        "e2e": {"value": round(tok_all * K_e2e / (e2e_ms_max / 1e3), 1), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "path": "pinned host qkv/offsets/cache_lengths/page_table -> device, "
+                        "rope_paged_kv_b200.rope_split_store_paged_ragged, q_out -> pinned host"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(), "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": alg,
+                     "kernel": "banded_store_kernel<bf16, 128, store>"},
+        "clocks": sampler.summary(t0, t1),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if extras:
+        line["entry_points"] = extras
+    print(json.dumps(line), flush=True)
+
+
+def time_launches(torch, launch, flush, reps=20, warm=3):
+    stream = torch.cuda.current_stream()
+    for _ in range(warm):
+        flush.zero_()
+        launch()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        launch()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / reps / 1e3  # seconds per launch
+
+
+def run_entry_points(rs, W, dev, flush):
+    """The other entry points on their named workloads (N=1 only; reported, not headline)."""
+    import torch
+
+    def d(t):
+        return t.to(dev)
+
+    def paged(kv, storage):
+        return rs.PagedCache(storage[kv.k_offset:],
+                             None if kv.v_offset is None else storage[kv.v_offset:],
+                             d(kv.page_table), d(kv.cache_lengths), kv.n_kv_heads,
+                             kv.head_dim, kv.page_size, kv.num_pages, kv.num_layers,
+                             kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride)
+
+    out = {}
+
+    def record(name, w, tokens, nbytes, sec):
+        out[name] = {"workload": w.name, "tokens": tokens, "us_per_launch": round(sec * 1e6, 2),
+                     "tokens_per_s": round(tokens / sec, 1),
+                     "algorithmic_gbs": round(nbytes / sec / 1e9, 1)}
+
+    w = W.per_head_norm()
+    st, qo = d(w.cache.storage), d(w.q_out)
+    args = (d(w.qkv), w.n_q_heads, d(w.offsets), rs.Freqs(d(w.rope.table), w.rope.interleaved),
+            paged(w.cache, st), d(w.q_gamma), d(w.k_gamma), w.epsilon, w.weight_offset,
+            w.layer_idx, qo)
+    sec = time_launches(torch, lambda: rs.fused_qk_rmsnorm_rope_paged(*args), flush)
+    record("fused_qk_rmsnorm_rope_paged", w, w.total_tokens, bytes_ragged(w), sec)
+    del st, qo, args
+
+    w = W.dual_band_minimax()
+    inp = d(w.input)
+    ms, ist = d(w.main_cache.storage), d(w.index_cache.storage)
+    g = [d(x) for x in w.gammas]
+    main = rs.NormBand(inp, *w.main_cols, w.main_q_heads, paged(w.main_cache, ms), g[0], g[1],
+                       w.main_eps, d(w.q_main_out))
+    index = rs.NormBand(inp, *w.index_cols, w.index_q_heads, paged(w.index_cache, ist), g[2],
+                        g[3], w.index_eps, d(w.q_index_out))
+    offs, fr = d(w.offsets), rs.Freqs(d(w.rope.table), w.rope.interleaved)
+    sec = time_launches(torch, lambda: rs.fused_dual_qk_rmsnorm_rope_paged(
+        main, index, offs, w.total_tokens, fr, w.weight_offset, w.layer_idx), flush)
+    record("fused_dual_qk_rmsnorm_rope_paged", w, w.total_tokens, bytes_dual(w), sec)
+    del inp, ms, ist, main, index
+
+    w = W.radd_minimax()
+    st = d(w.cache.storage)
+    a, offs, kvr = d(w.a), d(w.offsets), None
+    kvr = paged(w.cache, st)
+    sec = time_launches(torch, lambda: rs.kv_cache_radd(a, kvr, offs, w.batch_offset,
+                                                        w.layer_idx), flush)
+    record("kv_cache_radd", w, w.a.shape[0], bytes_radd(w), sec)
+    del st, a, kvr
+
+    w = W.decode_bshd()
+    st, out_t = d(w.cache.storage), d(w.output)
+    kv = w.cache
+    cc = rs.ContCache(st, None, d(kv.lookup_table), d(kv.cache_lengths), kv.n_kv_heads,
+                      kv.head_dim, kv.num_slots, kv.num_layers, kv.max_seq_len, kv.slot_stride,
+                      kv.layer_stride, kv.pos_stride, kv.head_stride)
+    q, fr, vl = d(w.q_proj), rs.Freqs(d(w.rope.table), w.rope.interleaved), d(w.valid_lengths)
+    sec = time_launches(torch, lambda: rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl,
+                                                                  out_t), flush)
+    B, S = w.q_proj.shape[:2]
+    record("qk_rope_bshd_continuous", w, B * S, bytes_bshd(w), sec)
+    # back-to-back launches without the flush (the decode step's L2-warm case)
+    stream = torch.cuda.current_stream()
+    a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(3):
+        rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl, out_t)
+    a0.record(stream)
+    n = 50
+    for _ in range(n):
+        rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl, out_t)
+    b0.record(stream)
+    torch.cuda.synchronize()
+    out["qk_rope_bshd_continuous"]["us_per_launch_back_to_back_l2_warm"] = round(
+        a0.elapsed_time(b0) / n * 1e3, 2)
+    del st, out_t, cc, q
+    torch.cuda.empty_cache()
+    return out
+
+
+def cpu_baseline(W, min_seconds=10.0, max_reps=20):
+    """The oracle as it stands (single-threaded C, double precision) on the same workload."""
+    from oracle import runners as R
+    w = W.llama3_8b_prefill(seed=0)
+    reps, t_total = 0, 0.0
+    while t_total < min_seconds and reps < max_reps:
+        t = time.perf_counter()
+        R.oracle_ragged_store(w)
+        t_total += time.perf_counter() - t
+        reps += 1
+    return {"value": round(w.total_tokens * reps / t_total, 1), "unit": UNIT, "cores": 1,
+            "kind": "oracle",
+            "sample": f"the full benchmark batch ({w.total_tokens} tokens), {reps} passes, "
+                      f"{t_total:.1f} s; single-threaded C, double precision (host copy-in "
+                      f"of the arrays included)"}
+
+
+# --------------------------------------------------------------- reference arm --
+
+def run_reference(args):
+    """The CPU oracle timed on this workload (rank 0 only): the reference arm."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import workloads as W
+    from oracle import runners as R
+    full = W.llama3_8b_prefill(seed=0)
+    steps, warm = args.steps, max(3, args.warmup)
+    # size each step's sample of sequences so the whole run stays within ~2 minutes
+    t = time.perf_counter()
+    one = W.ragged_store(1, lengths=full.lengths[:1], cache_lengths=[0], n_q_heads=32,
+                         n_kv_heads=8, head_dim=128, page_size=128, rope_dim=128, theta=5e5,
+                         interleaved=False, max_seq_len=8192, width=64)
+    t = time.perf_counter()
+    R.oracle_ragged_store(one)
+    per_token = (time.perf_counter() - t) / one.total_tokens
+    budget = 120.0 / (steps + warm)
+    n_seq = 1
+    while n_seq < len(full.lengths) and sum(full.lengths[:n_seq + 1]) * per_token <= budget:
+        n_seq += 1
+    lengths = full.lengths[:n_seq]
+    w = W.ragged_store(1, lengths=lengths, cache_lengths=[0] * n_seq, n_q_heads=32,
+                       n_kv_heads=8, head_dim=128, page_size=128, rope_dim=128, theta=5e5,
+                       interleaved=False, max_seq_len=8192, width=64)
+    for _ in range(warm):
+        R.oracle_ragged_store(w)
+    total = 0.0
+    for _ in range(steps):
+        t = time.perf_counter()
+        R.oracle_ragged_store(w)
+        total += time.perf_counter() - t
+    value = w.total_tokens * steps / total
+    sample = (f"first {n_seq} of the 8 sequences ({w.total_tokens} tokens) per step; "
+              f"single-threaded C oracle, double precision")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm,
+        "ms_per_step": round(total / steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": full.name, "entry_point": "rope_split_store_paged_ragged",
+                   "sample": sample},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

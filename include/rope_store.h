@@ -1,0 +1,238 @@
+/*
+ * rope_store.h -- attention-prologue kernels for NVIDIA B200 (sm_100a): RoPE, per-head
+ * RMSNorm and paged / continuous K/V-cache stores, behind a plain C ABI.
+ *
+ * The operations follow five Modular MAX kernel reference pages; each entry point below
+ * names the page and the part of it that defines the operation.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every pointer argument is a device pointer owned by the caller (destination-
+ *           passing style: the caller allocates every output, as the pages' signatures do
+ *           for their output tensors).  Descriptor structs (rope_freqs_t, rope_paged_cache_t, ...) live in
+ *           host memory and are read only during the call.  The library allocates, frees
+ *           and synchronises nothing.
+ * Streams.  Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *           default stream).  Work on one stream runs in order, which is what orders a
+ *           store after the projection that produced its input.
+ * Layout.   Rows are token-major; strides are in ELEMENTS.  Within a row, heads are
+ *           contiguous blocks of head_dim elements.  All tensor base pointers, row strides
+ *           and column offsets must keep every head row 16-byte aligned.
+ * Types.    Element types: ROPE_DTYPE_BF16, ROPE_DTYPE_F16, ROPE_DTYPE_F32.  The cache uses
+ *           the input's element type.  freqs_cis may be F32, BF16 or F16.  head_dim is 64,
+ *           128 or 256 (64 or 128 for F32 elements).
+ * Math.     Values are widened to float32, normalised and rotated in float32, and rounded
+ *           once, to nearest even, into the output type.  V heads and columns that are
+ *           neither normalised nor rotated are copied bit for bit.
+ * Status.   The return value reports argument problems found on the host before any
+ *           launch (nothing is written then) and launch failures.  total_tokens == 0 (or
+ *           batch*seq_len == 0) returns ROPE_OK at once, without a launch and without
+ *           looking at the other arguments (empty tensors may have NULL data).
+ * Device errors.  Problems that depend on device data are found by the kernel: it ORs the
+ *           ROPE_DEVERR_* bits into *err_word (if err_word is not NULL) and skips the
+ *           affected token, writing none of its outputs; other tokens are unaffected.  If
+ *           input_row_offsets is not a partition of [0, total_tokens) (first entry 0,
+ *           non-decreasing, last entry total_tokens) the whole call writes nothing.  The
+ *           kernels never trap and never wait on other blocks.
+ */
+#ifndef ROPE_STORE_H
+#define ROPE_STORE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *rope_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  ROPE_OK = 0,
+  ROPE_ERR_INVALID_ARG = 1, /* NULL pointer, negative size, inconsistent geometry */
+  ROPE_ERR_UNSUPPORTED = 2, /* dtype / head_dim / rope geometry / alignment not supported */
+  ROPE_ERR_CUDA = 3         /* the launch failed (cudaGetLastError() has the cause) */
+} rope_status_t;
+
+typedef enum { ROPE_DTYPE_BF16 = 0, ROPE_DTYPE_F16 = 1, ROPE_DTYPE_F32 = 2 } rope_dtype_t;
+
+/* bits of *err_word */
+#define ROPE_DEVERR_ROW_OFFSETS 0x1u /* input_row_offsets is not a partition of [0, T) */
+#define ROPE_DEVERR_POSITION 0x2u    /* position >= rows of freqs_cis (or of the cache) */
+#define ROPE_DEVERR_PAGE_INDEX 0x4u  /* position / page_size >= max_pages_per_seq */
+#define ROPE_DEVERR_PAGE_ID 0x8u     /* page-table entry >= num_pages */
+#define ROPE_DEVERR_BATCH 0x10u      /* sequence (+ batch_offset) >= n_seqs, or slot >= num_slots */
+
+/* freqs_cis [max_seq_len, rope_dim], row-major, contiguous.  Row p holds rope_dim/2
+ * pairs (cos, sin): column 2i is cos and 2i+1 is sin of pair i's angle at position p (the
+ * table argument of the rope_split_store_paged_ragged page, Args, stores the two parts of
+ * each rotation next to each other).
+ * rope_dim = the table's column count (fused_dual_qk_rms_norm_rope_ragged_paged, second
+ * paragraph: rope_dim comes from freqs_cis's second dimension); it is even, at most
+ * head_dim, and rope_dim < head_dim means partial RoPE.
+ * interleaved != 0: pair i of a head is columns (o + 2i, o + 2i + 1): the real and
+ *   imaginary parts side by side (rope_split_store_paged_ragged, Parameters, interleaved);
+ * interleaved == 0: pair i is columns (o + i, o + i + rope_dim/2) (half-split layout).
+ * o = rope_col_offset, or head_dim - rope_dim when rope_col_offset < 0: partial RoPE
+ * rotates the last rope_dim columns of each head unless the caller says otherwise.
+ * Supported: o and rope_dim multiples of the 16-byte vector width (8 elements for 16-bit
+ * types, 4 for F32), and for the half-split layout rope_dim/2 too. */
+typedef struct {
+  const void *data;
+  int32_t dtype; /* rope_dtype_t of the table */
+  int32_t max_seq_len;
+  int32_t rope_dim;
+  int32_t interleaved;
+  int32_t rope_col_offset;
+} rope_freqs_t;
+
+/* A paged K/V cache (PagedKVCacheCollection on the pages).  Element (page, layer, slot,
+ * head, d) of the K plane is
+ *     k[page*page_stride + layer*layer_stride + slot*slot_stride + head*head_stride + d]
+ * and of the V plane likewise from v (v may be NULL for a K-only cache).  A sequence's
+ * position p lives in page page_table[seq*page_table_stride + p / page_size] at slot
+ * p % page_size.  cache_lengths[seq] = tokens the sequence already holds; new token t of
+ * the sequence goes to position cache_lengths[seq] + t.  page_table and cache_lengths are
+ * device arrays with n_seqs rows. */
+typedef struct {
+  void *k;
+  void *v;
+  int32_t dtype;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t num_pages;
+  int32_t num_layers;
+  int64_t page_stride, layer_stride, slot_stride, head_stride; /* elements */
+  const uint32_t *page_table;
+  int64_t page_table_stride; /* elements between consecutive sequences' rows */
+  int32_t max_pages_per_seq; /* usable entries of a page-table row */
+  const uint32_t *cache_lengths;
+  int32_t n_seqs;
+} rope_paged_cache_t;
+
+/* A continuous-batching K/V cache (ContinuousBatchingKVCacheCollection on the pages).
+ * Batch entry b owns slot lookup_table[b]; element (slot, layer, pos, head, d) of the K
+ * plane is k[slot*slot_stride + layer*layer_stride + pos*pos_stride + head*head_stride + d].
+ * lookup_table and cache_lengths are device arrays with n_seqs entries. */
+typedef struct {
+  void *k;
+  void *v;
+  int32_t dtype;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t num_slots;
+  int32_t num_layers;
+  int32_t max_seq_len;
+  int64_t slot_stride, layer_stride, pos_stride, head_stride; /* elements */
+  const uint32_t *lookup_table;
+  const uint32_t *cache_lengths;
+  int32_t n_seqs;
+} rope_cont_cache_t;
+
+/* One band of the dual per-head RMSNorm + RoPE launch: its Q heads start at column q_col,
+ * its K heads at k_col and its V heads at v_col (v_col < 0: the band's cache is K-only) of
+ * the token-major `input` (the pages' per-band Q read lambdas become a base pointer, a row
+ * stride and column offsets).  q_gamma / k_gamma: [head_dim] in the element type, shared by
+ * all Q (K) heads of the band.  epsilon: the band's RMSNorm epsilon.  q_out: [T, n_q_heads *
+ * head_dim] rows with stride q_out_row_stride. */
+typedef struct {
+  const void *input;
+  int64_t input_row_stride;
+  int64_t q_col, k_col, v_col;
+  int32_t n_q_heads;
+  const rope_paged_cache_t *cache;
+  const void *q_gamma;
+  const void *k_gamma;
+  float epsilon;
+  void *q_out;
+  int64_t q_out_row_stride;
+} rope_norm_band_t;
+
+/* rope_split_store_paged_ragged -- rotate Q and K of a flat ragged QKV batch, write Q
+ * out and store K and V into a paged cache (rope_split_store_paged_ragged page: signature,
+ * Parameters, Args).
+ *   qkv [total_tokens, (n_q_heads + 2*n_kv_heads) * head_dim], row stride qkv_row_stride:
+ *       the flat matmul output, columns Q | K | V.
+ *   input_row_offsets [batch + 1]: sequence b owns rows [offs[b], offs[b+1]).
+ *   Row r of sequence b sits at position p = kv->cache_lengths[b] + (r - offs[b]).
+ *   Q heads are rotated with freqs_cis row p and written to q_out [total_tokens, n_q_heads *
+ *   head_dim] (row stride q_out_row_stride); K heads are rotated and V heads copied into the
+ *   cache of layer layer_idx at position p.  kv->v must not be NULL. */
+rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_stride,
+                                            int32_t total_tokens, int32_t n_q_heads,
+                                            const uint32_t *input_row_offsets, int32_t batch,
+                                            const rope_freqs_t *freqs,
+                                            const rope_paged_cache_t *kv, uint32_t layer_idx,
+                                            void *q_out, int64_t q_out_row_stride,
+                                            uint32_t *err_word, rope_stream_t stream);
+
+/* fused_qk_rmsnorm_rope_paged -- the single-band per-head RMSNorm + RoPE + paged store that
+ * the fused_dual_qk_rms_norm_rope_ragged_paged page fuses twice (its first paragraph).
+ * As rope_split_store_paged_ragged, but each Q (K) head row x of head_dim elements first
+ * becomes x * rsqrt(mean(x^2) + epsilon) * (gamma + weight_offset) with gamma = q_gamma
+ * (k_gamma); RoPE then rotates that normalised row (no rounding in between).
+ * weight_offset is a scalar of the element type (the page's Scalar[dtype]): it is rounded
+ * to the element type first.  multiply_before_cast must be 1 (the normalised row is
+ * multiplied by gamma before any rounding); 0 returns ROPE_ERR_UNSUPPORTED. */
+rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_stride,
+                                          int32_t total_tokens, int32_t n_q_heads,
+                                          const uint32_t *input_row_offsets, int32_t batch,
+                                          const rope_freqs_t *freqs,
+                                          const rope_paged_cache_t *kv, const void *q_gamma,
+                                          const void *k_gamma, float epsilon,
+                                          float weight_offset, int32_t multiply_before_cast,
+                                          uint32_t layer_idx, void *q_out,
+                                          int64_t q_out_row_stride, uint32_t *err_word,
+                                          rope_stream_t stream);
+
+/* fused_dual_qk_rmsnorm_rope_paged -- fused_dual_qk_rms_norm_rope_ragged_paged page
+ * (signature and both paragraphs): the main band and the index band in ONE launch.  Both
+ * bands share input_row_offsets, total_tokens, freqs_cis, weight_offset,
+ * multiply_before_cast and layer_idx; each has its own input columns, cache, gammas,
+ * epsilon and Q output, and each band's positions come from its own cache_lengths.  The
+ * rope geometry must agree across bands: same element type and head_dim in both caches
+ * (else ROPE_ERR_INVALID_ARG, the runtime form of the page's compile-time assert).  The
+ * result equals fused_qk_rmsnorm_rope_paged on the main band followed by the same on the
+ * index band. */
+rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band,
+                                               const rope_norm_band_t *index_band,
+                                               const uint32_t *input_row_offsets,
+                                               int32_t batch, int32_t total_tokens,
+                                               const rope_freqs_t *freqs, float weight_offset,
+                                               int32_t multiply_before_cast, uint32_t layer_idx,
+                                               uint32_t *err_word, rope_stream_t stream);
+
+/* qk_rope_bshd_continuous -- generic_fused_qk_rope_bshd_continuous_batch page (signature,
+ * description, Args).  q_proj and output: [batch, seq_len, n_q_heads, head_dim],
+ * contiguous.  For s < valid_lengths[b] (device array [batch]): position p =
+ * kv->cache_lengths[b] + s; Q head rows are rotated with freqs_cis row p into output, and
+ * the K head rows at (kv->lookup_table[b], layer_idx, p) are rotated IN PLACE in the cache.
+ * For s >= valid_lengths[b]: output = q_proj unchanged and the cache is not touched.
+ * p must be below both freqs->max_seq_len and kv->max_seq_len (else ROPE_DEVERR_POSITION
+ * and the token is skipped). */
+rope_status_t qk_rope_bshd_continuous(const void *q_proj, int32_t batch, int32_t seq_len,
+                                      int32_t n_q_heads, int32_t head_dim,
+                                      const rope_cont_cache_t *kv, const rope_freqs_t *freqs,
+                                      uint32_t layer_idx, const uint32_t *valid_lengths,
+                                      void *output, uint32_t *err_word, rope_stream_t stream);
+
+/* kv_cache_radd -- generic_kv_cache_radd_dispatch page (description, Args).  a
+ * [total_tokens, 2 * n_kv_heads * head_dim], row stride a_row_stride: the first
+ * n_kv_heads*head_dim columns are added into K, the rest into V.  Row r of sequence b
+ * targets cache sequence b' = b + batch_offset at position kv->cache_lengths[b'] +
+ * (r - offs[b]) of layer layer_idx.  Each cache element becomes the float32 sum rounded
+ * once to the element type (for 16-bit types this equals the correctly rounded exact sum).
+ * kv->v must not be NULL. */
+rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_tokens,
+                            const rope_paged_cache_t *kv, const uint32_t *input_row_offsets,
+                            int32_t batch, uint32_t batch_offset, uint32_t layer_idx,
+                            uint32_t *err_word, rope_stream_t stream);
+
+/* A static, human-readable name of a status code. */
+const char *rope_status_string(rope_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ROPE_STORE_H */

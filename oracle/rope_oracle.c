@@ -7,19 +7,22 @@
  *   [P1] "generic_fused_qk_rope_bshd_continuous_batch": description paragraph and Args
  *        (q_proj [batch, seq_len, n_heads, head_dim]; valid_lengths: RoPE only for positions
  *        inside the valid length; output same shape as q_proj).
- *   [P2] "rope_split_store_paged_ragged": "Rope+split+store"; Args qkv = flat matmul output
- *        [total_seq_len, q_dim + k_dim + v_dim], input_row_offsets [batch_size + 1],
- *        freqs_cis [max_seq_len, head_dim] interleaved frequencies, q_output
- *        [total_seq_len, q_dim]; Parameters: interleaved (real/imag layout).
- *   [P3] "generic_kv_cache_radd_dispatch": description and Args (a [sum(seq_lens),
- *        2*hidden_size], first hidden_size columns to K, rest to V; batch_offset added to the
- *        computed batch index; per-batch cache lengths locate the target rows).
+ *   [P2] "rope_split_store_paged_ragged": one-line description (rotate, split the QKV
+ *        columns, store into the paged cache); Args: qkv is the flat projection output
+ *        [total_seq_len, q_dim + k_dim + v_dim], input_row_offsets has batch_size + 1
+ *        entries, freqs_cis is [max_seq_len, head_dim] with the two parts of each rotation
+ *        side by side, q_output is [total_seq_len, q_dim]; Parameters: interleaved (layout of
+ *        the rotated pairs).
+ *   [P3] "generic_kv_cache_radd_dispatch": description and Args (a is [sum(seq_lens),
+ *        2*hidden_size]; its first half of columns goes to K and its second half to V; the
+ *        batch index is shifted by batch_offset; the cache length of the sequence gives the
+ *        row's position).
  *   [P4] "fused_dual_qk_rms_norm_rope_ragged_paged": signature (gammas, main/index epsilon,
  *        weight_offset, multiply_before_cast) and both description paragraphs (one launch
  *        equals two single-band fused_qk_rms_norm_rope_ragged_paged launches; rope geometry
  *        identical across bands; rope_dim = columns of freqs_cis).
- *   [P5] "MatmulFusedPartialRMSNorm": Args, epsilon is added to the mean square before the
- *        reciprocal square root.
+ *   [P5] "MatmulFusedPartialRMSNorm": Args (epsilon sits inside the inverse square root,
+ *        with the mean of squares).
  *
  * Readings chosen where the pages leave a step open:
  *   - freqs_cis row p = (cos, sin) pairs of pair i at columns 2i, 2i+1, for both layouts;

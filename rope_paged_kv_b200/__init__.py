@@ -1,0 +1,292 @@
+"""Python binding of ``librope_store.so`` (include/rope_store.h): argument marshalling only.
+
+Every function takes torch CUDA tensors (for memory) and an optional torch CUDA stream,
+builds the C descriptors from their data pointers and calls the C entry point of the same
+name.  All arithmetic runs in the library's sm_100a kernels; there is no fallback, and a
+missing library raises at import time.
+
+Descriptors
+-----------
+Freqs(table, interleaved, rope_col_offset=-1)
+    freqs_cis [max_seq_len, rope_dim] (f32 / bf16 / f16): (cos, sin) of pair i at columns
+    2i, 2i+1.  rope_col_offset: first rotated column of a head (-1 = head_dim - rope_dim).
+PagedCache(k, v, page_table, cache_lengths, n_kv_heads, head_dim, page_size, num_pages,
+           num_layers, page_stride, layer_stride, slot_stride, head_stride)
+    k / v: tensors whose data pointers are the K / V plane bases (v may be None for a K-only
+    cache); strides in elements; page_table int32/uint32 [n_seqs, width]; cache_lengths
+    [n_seqs].
+ContCache(k, v, lookup_table, cache_lengths, n_kv_heads, head_dim, num_slots, num_layers,
+          max_seq_len, slot_stride, layer_stride, pos_stride, head_stride)
+NormBand(input, q_col, k_col, v_col, n_q_heads, cache, q_gamma, k_gamma, epsilon, q_out)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_PKG, "librope_store.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "rope_store.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA = 0, 1, 2, 3
+DEVERR_ROW_OFFSETS, DEVERR_POSITION, DEVERR_PAGE_INDEX = 0x1, 0x2, 0x4
+DEVERR_PAGE_ID, DEVERR_BATCH = 0x8, 0x10
+
+_DTYPE_CODE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+
+if not os.path.exists(LIBRARY_PATH):
+    raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
+                      f"`python -m rope_paged_kv_b200.build` (nvcc, sm_100a)")
+_lib = ctypes.CDLL(LIBRARY_PATH)
+
+_vp, _i32, _i64, _u32, _f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                               ctypes.c_uint32, ctypes.c_float)
+
+
+class c_freqs(ctypes.Structure):
+    _fields_ = [("data", _vp), ("dtype", _i32), ("max_seq_len", _i32), ("rope_dim", _i32),
+                ("interleaved", _i32), ("rope_col_offset", _i32)]
+
+
+class c_paged_cache(ctypes.Structure):
+    _fields_ = [("k", _vp), ("v", _vp), ("dtype", _i32), ("n_kv_heads", _i32),
+                ("head_dim", _i32), ("page_size", _i32), ("num_pages", _i32),
+                ("num_layers", _i32), ("page_stride", _i64), ("layer_stride", _i64),
+                ("slot_stride", _i64), ("head_stride", _i64), ("page_table", _vp),
+                ("page_table_stride", _i64), ("max_pages_per_seq", _i32),
+                ("cache_lengths", _vp), ("n_seqs", _i32)]
+
+
+class c_cont_cache(ctypes.Structure):
+    _fields_ = [("k", _vp), ("v", _vp), ("dtype", _i32), ("n_kv_heads", _i32),
+                ("head_dim", _i32), ("num_slots", _i32), ("num_layers", _i32),
+                ("max_seq_len", _i32), ("slot_stride", _i64), ("layer_stride", _i64),
+                ("pos_stride", _i64), ("head_stride", _i64), ("lookup_table", _vp),
+                ("cache_lengths", _vp), ("n_seqs", _i32)]
+
+
+class c_norm_band(ctypes.Structure):
+    _fields_ = [("input", _vp), ("input_row_stride", _i64), ("q_col", _i64), ("k_col", _i64),
+                ("v_col", _i64), ("n_q_heads", _i32), ("cache", ctypes.POINTER(c_paged_cache)),
+                ("q_gamma", _vp), ("k_gamma", _vp), ("epsilon", _f32), ("q_out", _vp),
+                ("q_out_row_stride", _i64)]
+
+
+_P = ctypes.POINTER
+_lib.rope_split_store_paged_ragged.argtypes = [
+    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp, _vp]
+_lib.fused_qk_rmsnorm_rope_paged.argtypes = [
+    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _vp, _vp, _f32, _f32,
+    _i32, _u32, _vp, _i64, _vp, _vp]
+_lib.fused_dual_qk_rmsnorm_rope_paged.argtypes = [
+    _P(c_norm_band), _P(c_norm_band), _vp, _i32, _i32, _P(c_freqs), _f32, _i32, _u32, _vp, _vp]
+_lib.qk_rope_bshd_continuous.argtypes = [
+    _vp, _i32, _i32, _i32, _i32, _P(c_cont_cache), _P(c_freqs), _u32, _vp, _vp, _vp, _vp]
+_lib.kv_cache_radd.argtypes = [
+    _vp, _i64, _i32, _P(c_paged_cache), _vp, _i32, _u32, _u32, _vp, _vp]
+for _f in ("rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
+           "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd"):
+    getattr(_lib, _f).restype = ctypes.c_int
+_lib.rope_status_string.argtypes = [ctypes.c_int]
+_lib.rope_status_string.restype = ctypes.c_char_p
+
+
+def header_functions() -> list:
+    """Names of the functions include/rope_store.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"^(?:rope_status_t|const char \*)\s*\n?\s*\**(\w+)\(", text, re.M)
+
+
+class RopeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.rope_status_string(status).decode()} "
+                         f"(status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise RopeError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _row_stride(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with contiguous rows")
+    return t.stride(0)
+
+
+def _idx(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype not in (torch.int32, torch.uint32) or not t.is_contiguous():
+        raise ValueError("index arrays must be contiguous int32/uint32")
+    return t
+
+
+@dataclass
+class Freqs:
+    table: torch.Tensor
+    interleaved: bool
+    rope_col_offset: int = -1
+
+    def c(self) -> c_freqs:
+        t = self.table
+        if t.dim() != 2 or not t.is_contiguous():
+            raise ValueError("freqs_cis must be a contiguous [max_seq_len, rope_dim] tensor")
+        return c_freqs(t.data_ptr(), _DTYPE_CODE[t.dtype], t.shape[0], t.shape[1],
+                       int(bool(self.interleaved)), self.rope_col_offset)
+
+
+@dataclass
+class PagedCache:
+    k: torch.Tensor
+    v: Optional[torch.Tensor]
+    page_table: torch.Tensor
+    cache_lengths: torch.Tensor
+    n_kv_heads: int
+    head_dim: int
+    page_size: int
+    num_pages: int
+    num_layers: int
+    page_stride: int
+    layer_stride: int
+    slot_stride: int
+    head_stride: int
+    max_pages_per_seq: Optional[int] = None
+
+    def c(self) -> c_paged_cache:
+        pt = _idx(self.page_table)
+        width = pt.shape[1] if self.max_pages_per_seq is None else self.max_pages_per_seq
+        return c_paged_cache(self.k.data_ptr(), _ptr(self.v), _DTYPE_CODE[self.k.dtype],
+                             self.n_kv_heads, self.head_dim, self.page_size, self.num_pages,
+                             self.num_layers, self.page_stride, self.layer_stride,
+                             self.slot_stride, self.head_stride, pt.data_ptr(), pt.stride(0),
+                             width, _idx(self.cache_lengths).data_ptr(), pt.shape[0])
+
+
+@dataclass
+class ContCache:
+    k: torch.Tensor
+    v: Optional[torch.Tensor]
+    lookup_table: torch.Tensor
+    cache_lengths: torch.Tensor
+    n_kv_heads: int
+    head_dim: int
+    num_slots: int
+    num_layers: int
+    max_seq_len: int
+    slot_stride: int
+    layer_stride: int
+    pos_stride: int
+    head_stride: int
+
+    def c(self) -> c_cont_cache:
+        lt = _idx(self.lookup_table)
+        return c_cont_cache(self.k.data_ptr(), _ptr(self.v), _DTYPE_CODE[self.k.dtype],
+                            self.n_kv_heads, self.head_dim, self.num_slots, self.num_layers,
+                            self.max_seq_len, self.slot_stride, self.layer_stride,
+                            self.pos_stride, self.head_stride, lt.data_ptr(),
+                            _idx(self.cache_lengths).data_ptr(), lt.shape[0])
+
+
+@dataclass
+class NormBand:
+    input: torch.Tensor
+    q_col: int
+    k_col: int
+    v_col: int
+    n_q_heads: int
+    cache: PagedCache
+    q_gamma: torch.Tensor
+    k_gamma: torch.Tensor
+    epsilon: float
+    q_out: torch.Tensor
+
+    def c(self, keep: list) -> c_norm_band:
+        pc = self.cache.c()
+        keep.append(pc)
+        return c_norm_band(self.input.data_ptr(), _row_stride(self.input), self.q_col,
+                           self.k_col, self.v_col, self.n_q_heads, ctypes.pointer(pc),
+                           self.q_gamma.data_ptr(), self.k_gamma.data_ptr(), self.epsilon,
+                           self.q_out.data_ptr(), _row_stride(self.q_out))
+
+
+# ------------------------------------------------------------------------ entry points --
+
+def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
+                                  kv: PagedCache, layer_idx, q_out, err_word=None,
+                                  stream=None) -> None:
+    offs = _idx(input_row_offsets)
+    f, c = freqs.c(), kv.c()
+    _check(_lib.rope_split_store_paged_ragged(
+        qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
+        offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
+        _row_stride(q_out), _ptr(err_word), _stream(stream)), "rope_split_store_paged_ragged")
+
+
+def fused_qk_rmsnorm_rope_paged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
+                                kv: PagedCache, q_gamma, k_gamma, epsilon, weight_offset,
+                                layer_idx, q_out, multiply_before_cast=True, err_word=None,
+                                stream=None) -> None:
+    offs = _idx(input_row_offsets)
+    f, c = freqs.c(), kv.c()
+    _check(_lib.fused_qk_rmsnorm_rope_paged(
+        qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
+        offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), q_gamma.data_ptr(),
+        k_gamma.data_ptr(), epsilon, weight_offset, int(bool(multiply_before_cast)), layer_idx,
+        q_out.data_ptr(), _row_stride(q_out), _ptr(err_word), _stream(stream)),
+        "fused_qk_rmsnorm_rope_paged")
+
+
+def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: NormBand,
+                                     input_row_offsets, total_tokens, freqs: Freqs,
+                                     weight_offset, layer_idx, multiply_before_cast=True,
+                                     err_word=None, stream=None) -> None:
+    offs = _idx(input_row_offsets)
+    keep: list = []
+    m, i, f = main_band.c(keep), index_band.c(keep), freqs.c()
+    _check(_lib.fused_dual_qk_rmsnorm_rope_paged(
+        ctypes.byref(m), ctypes.byref(i), offs.data_ptr(), offs.shape[0] - 1, total_tokens,
+        ctypes.byref(f), weight_offset, int(bool(multiply_before_cast)), layer_idx,
+        _ptr(err_word), _stream(stream)), "fused_dual_qk_rmsnorm_rope_paged")
+
+
+def qk_rope_bshd_continuous(q_proj, kv: ContCache, freqs: Freqs, layer_idx, valid_lengths,
+                            output, err_word=None, stream=None) -> None:
+    if q_proj.dim() != 4 or not q_proj.is_contiguous() or not output.is_contiguous():
+        raise ValueError("q_proj / output must be contiguous [batch, seq_len, heads, head_dim]")
+    B, S, H, D = q_proj.shape
+    c, f = kv.c(), freqs.c()
+    _check(_lib.qk_rope_bshd_continuous(
+        q_proj.data_ptr(), B, S, H, D, ctypes.byref(c), ctypes.byref(f), layer_idx,
+        _idx(valid_lengths).data_ptr(), output.data_ptr(), _ptr(err_word), _stream(stream)),
+        "qk_rope_bshd_continuous")
+
+
+def kv_cache_radd(a, kv: PagedCache, input_row_offsets, batch_offset, layer_idx,
+                  err_word=None, stream=None) -> None:
+    offs = _idx(input_row_offsets)
+    c = kv.c()
+    _check(_lib.kv_cache_radd(
+        a.data_ptr(), _row_stride(a), a.shape[0], ctypes.byref(c), offs.data_ptr(),
+        offs.shape[0] - 1, batch_offset, layer_idx, _ptr(err_word), _stream(stream)),
+        "kv_cache_radd")
+
+
+def raw_library() -> ctypes.CDLL:
+    """The loaded C library, for callers that pass raw pointers themselves."""
+    return _lib

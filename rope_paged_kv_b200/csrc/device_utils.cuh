@@ -1,0 +1,95 @@
+// device_utils.cuh -- 16-byte element vectors and small helpers for the prologue kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rs {
+
+// A 16-byte vector of N elements of type T, widened to / narrowed from float32.
+template <typename T>
+struct Vec;
+
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  static __device__ __forceinline__ void widen(const uint4 v, float (&x)[N]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);              // low half = lower address
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);  // bf16 is the top of an f32
+    }
+  }
+  static __device__ __forceinline__ uint4 narrow(const float (&x)[N]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+template <>
+struct Vec<__half> {
+  static constexpr int N = 8;
+  static __device__ __forceinline__ void widen(const uint4 v, float (&x)[N]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+      float2 f = __half22float2(h);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ uint4 narrow(const float (&x)[N]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  static __device__ __forceinline__ void widen(const uint4 v, float (&x)[N]) {
+    x[0] = __uint_as_float(v.x);
+    x[1] = __uint_as_float(v.y);
+    x[2] = __uint_as_float(v.z);
+    x[3] = __uint_as_float(v.w);
+  }
+  static __device__ __forceinline__ uint4 narrow(const float (&x)[N]) {
+    return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
+                      __float_as_uint(x[3]));
+  }
+};
+
+// One element of a freqs_cis table of runtime type (0 = bf16, 1 = f16, 2 = f32).
+__device__ __forceinline__ float load_freq(const void *table, int dtype, int64_t i) {
+  if (dtype == 2) return __ldg(reinterpret_cast<const float *>(table) + i);
+  const unsigned short b = __ldg(reinterpret_cast<const unsigned short *>(table) + i);
+  if (dtype == 0) return __uint_as_float(static_cast<uint32_t>(b) << 16);
+  return __half2float(__ushort_as_half(b));
+}
+
+// Streaming (read-once) 16-byte load and plain 16-byte store.
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+  return __ldcs(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ uint4 ld_plain(const void *p) {
+  return *reinterpret_cast<const uint4 *>(p);
+}
+__device__ __forceinline__ void st_plain(void *p, uint4 v) {
+  *reinterpret_cast<uint4 *>(p) = v;
+}
+
+}  // namespace rs

@@ -12,16 +12,9 @@ import oracle
 import workloads as W
 
 
-def bits(t: torch.Tensor) -> np.ndarray:
-    """A host copy of a tensor's raw element bits (uint16 for 16-bit types)."""
-    t = t.detach().cpu().contiguous()
-    if t.dtype in (torch.bfloat16, torch.float16):
-        return t.view(torch.int16).numpy().view(np.uint16).copy()
-    if t.dtype == torch.float32:
-        return t.numpy().copy()
-    if t.dtype == torch.int32:
-        return t.numpy().view(np.uint32).copy()
-    raise TypeError(t.dtype)
+from oracle.runners import (bits, oracle_rope, oracle_paged, oracle_cont,  # noqa: F401
+                            OracleResult, oracle_ragged_store, oracle_dual, oracle_bshd,
+                            oracle_radd)
 
 
 def values(b: np.ndarray, dtype: str) -> np.ndarray:
@@ -31,90 +24,6 @@ def values(b: np.ndarray, dtype: str) -> np.ndarray:
     if dtype == "f16":
         return b.view(np.float16).astype(np.float64)
     return torch.from_numpy(b.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
-
-
-def oracle_rope(r: W.RopeSpec) -> oracle.Rope:
-    return oracle.Rope(bits(r.table), r.dtype, r.interleaved, r.rope_col_offset)
-
-
-def oracle_paged(kv: W.PagedKV, storage: np.ndarray) -> oracle.PagedCache:
-    return oracle.PagedCache(storage, kv.k_offset, kv.v_offset, kv.dtype, kv.n_kv_heads,
-                             kv.head_dim, kv.page_size, kv.num_pages, kv.num_layers,
-                             kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride,
-                             bits(kv.page_table), kv.max_pages_per_seq, bits(kv.cache_lengths))
-
-
-def oracle_cont(kv: W.ContKV, storage: np.ndarray) -> oracle.ContCache:
-    return oracle.ContCache(storage, kv.k_offset, kv.v_offset, kv.dtype, kv.n_kv_heads,
-                            kv.head_dim, kv.num_slots, kv.num_layers, kv.max_seq_len,
-                            kv.slot_stride, kv.layer_stride, kv.pos_stride, kv.head_stride,
-                            bits(kv.lookup_table), bits(kv.cache_lengths))
-
-
-class OracleResult(dict):
-    """Named host arrays the oracle produced (element bits) plus its error bits."""
-
-    def __getattr__(self, k):
-        return self[k]
-
-
-def oracle_ragged_store(w: W.RaggedStore, dtype: str = "bf16",
-                        multiply_before_cast: bool = True) -> OracleResult:
-    """The oracle on a ragged store workload: no-norm op when the workload has no gammas,
-    else the single-band norm op."""
-    store = bits(w.cache.storage)
-    q_out = bits(w.q_out)
-    qkv = bits(w.qkv)
-    written = np.zeros(w.cache.num_pages * w.cache.page_size, dtype=np.uint8)
-    cache = oracle_paged(w.cache, store)
-    rope = oracle_rope(w.rope)
-    if w.q_gamma is None:
-        err = oracle.rope_split_store_paged_ragged(qkv, w.n_q_heads, bits(w.offsets), rope,
-                                                   cache, w.layer_idx, q_out, written, dtype)
-    else:
-        D = w.cache.head_dim
-        Hq, Hk = w.n_q_heads, w.cache.n_kv_heads
-        band = oracle.Band(qkv, 0, Hq * D, (Hq + Hk) * D, Hq, cache, bits(w.q_gamma),
-                           bits(w.k_gamma), w.epsilon, q_out, written)
-        err = oracle.fused_qk_rmsnorm_rope_paged(band, bits(w.offsets), rope, w.weight_offset,
-                                                 multiply_before_cast, w.layer_idx, dtype)
-    return OracleResult(q_out=q_out, storage=store, written=written, err=err)
-
-
-def oracle_dual(w: W.DualBand, dtype: str = "bf16") -> OracleResult:
-    inp = bits(w.input)
-    ms, ist = bits(w.main_cache.storage), bits(w.index_cache.storage)
-    qm, qi = bits(w.q_main_out), bits(w.q_index_out)
-    wm = np.zeros(w.main_cache.num_pages * w.main_cache.page_size, dtype=np.uint8)
-    wi = np.zeros(w.index_cache.num_pages * w.index_cache.page_size, dtype=np.uint8)
-    g = [bits(x) for x in w.gammas]
-    main = oracle.Band(inp, *w.main_cols, w.main_q_heads, oracle_paged(w.main_cache, ms), g[0],
-                       g[1], w.main_eps, qm, wm)
-    index = oracle.Band(inp, *w.index_cols, w.index_q_heads, oracle_paged(w.index_cache, ist),
-                        g[2], g[3], w.index_eps, qi, wi)
-    err = oracle.fused_dual_qk_rmsnorm_rope_paged(main, index, bits(w.offsets),
-                                                  oracle_rope(w.rope), w.weight_offset, True,
-                                                  w.layer_idx, dtype)
-    return OracleResult(q_main_out=qm, q_index_out=qi, main_storage=ms, index_storage=ist,
-                        main_written=wm, index_written=wi, err=err)
-
-
-def oracle_bshd(w: W.BshdDecode, dtype: str = "bf16") -> OracleResult:
-    store = bits(w.cache.storage)
-    out = bits(w.output)
-    written = np.zeros(w.cache.num_slots * w.cache.max_seq_len, dtype=np.uint8)
-    err = oracle.qk_rope_bshd_continuous(bits(w.q_proj), oracle_cont(w.cache, store),
-                                         oracle_rope(w.rope), w.layer_idx,
-                                         bits(w.valid_lengths), out, written, dtype)
-    return OracleResult(output=out, storage=store, written=written, err=err)
-
-
-def oracle_radd(w: W.Radd, dtype: str = "bf16") -> OracleResult:
-    store = bits(w.cache.storage)
-    written = np.zeros(w.cache.num_pages * w.cache.page_size, dtype=np.uint8)
-    err = oracle.kv_cache_radd(bits(w.a), oracle_paged(w.cache, store), bits(w.offsets),
-                               w.batch_offset, w.layer_idx, written, dtype)
-    return OracleResult(storage=store, written=written, err=err)
 
 
 # ----------------------------------------------------------------------- comparisons --
@@ -141,16 +50,23 @@ def assert_close_bf16(got_bits: np.ndarray, want_bits: np.ndarray, what: str,
     else:
         ulp = np.spacing(np.abs(w).astype(np.float32)).astype(np.float64)
     tol = np.maximum(ulp, abs_tol)
-    bad = ~(np.abs(g - w) <= tol)
+    same = _as_bits(np.ascontiguousarray(got_bits)) == _as_bits(np.ascontiguousarray(want_bits))
+    bad = ~(same | (np.abs(g - w) <= tol))
     if bad.any():
         idx = np.argwhere(bad)[:8]
         raise AssertionError(
             f"{what}: {int(bad.sum())} of {bad.size} elements outside max(1 ulp, {abs_tol}); "
             f"first at {idx.tolist()}: got {g[bad][:8].tolist()} want {w[bad][:8].tolist()}")
-    return float((got_bits == want_bits).mean()) if got_bits.size else 1.0
+    return float((_as_bits(np.ascontiguousarray(got_bits)) ==
+                  _as_bits(np.ascontiguousarray(want_bits))).mean()) if got_bits.size else 1.0
+
+
+def _as_bits(a: np.ndarray) -> np.ndarray:
+    return a.view(np.uint32) if a.dtype == np.float32 else a
 
 
 def assert_bits_equal(got: np.ndarray, want: np.ndarray, what: str):
+    got, want = _as_bits(np.ascontiguousarray(got)), _as_bits(np.ascontiguousarray(want))
     if not np.array_equal(got, want):
         diff = np.argwhere(got != want)
         raise AssertionError(f"{what}: {len(diff)} elements differ; first at "
@@ -229,3 +145,37 @@ def golden_problem(case: dict, norm: bool, dtype: str = "bf16") -> W.RaggedStore
                          q_out, [1], g, None if g is None else g.clone(),
                          case.get("eps", 1e-6), case.get("weight_offset", 0.0),
                          case["name"])
+
+
+def tile_golden(case: dict, head_dim: int = 64) -> dict:
+    """The same worked example on a wider head: the pass-through columns and the rotated
+    columns are each repeated until the head is `head_dim` wide, keeping every rotation
+    pair's partner and (cos, sin) entry, so the expected row is the same repetition of the
+    expected values.  With no pass-through columns the mean square is unchanged too."""
+    D0, R0 = case["head_dim"], case["rope_dim"]
+    o0 = D0 - R0
+    R = head_dim if o0 == 0 else head_dim // 2
+    o = head_dim - R
+    rep_r = R // R0
+    assert rep_r * R0 == R and (o0 == 0 or (o // o0) * o0 == o)
+
+    def tile_row(x):
+        x = list(x)
+        head = (x[:o0] * (o // o0)) if o0 else []
+        rot = x[o0:]
+        if case["interleaved"]:
+            tail = rot * rep_r
+        else:
+            h = R0 // 2
+            tail = rot[:h] * rep_r + rot[h:] * rep_r
+        return head + tail
+
+    c = dict(case)
+    c["head_dim"], c["rope_dim"] = head_dim, R
+    c["x"] = tile_row(case["x"])
+    c["expect"] = tile_row(case["expect"])
+    c["freqs_row"] = list(case["freqs_row"]) * rep_r
+    if "gamma" in case:
+        assert o0 == 0
+        c["gamma"] = tile_row(case["gamma"])
+    return c

@@ -92,6 +92,16 @@ def test_rmsnorm_worked_examples(case):
     assert v.tolist() == list(range(1, case["head_dim"] + 1))
 
 
+@pytest.mark.parametrize("fname,norm", [("rope_worked_examples.json", False),
+                                         ("rmsnorm_worked_examples.json", True)])
+def test_worked_examples_tiled_to_head_dim_64(fname, norm):
+    for case in _golden(fname)["cases"]:
+        c = H.tile_golden(case, 64)
+        q, k, v, _ = _run_golden(c, norm)
+        assert q.tolist() == c["expect"], case["name"]
+        assert k.tolist() == c["expect"], case["name"]
+
+
 def _placement_problem(g, D=8, Hq=1, Hk=1, seed=11):
     gen = W.generator(seed)
     T = sum(g["lengths"])
