@@ -38,7 +38,8 @@ METRIC = "fused RoPE+KV-store tokens/s and achieved HBM GB/s (% of B200 peak), 1
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/rope_store.cu",
+KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/rope_store.cu", "rope_paged_kv_b200/csrc/banded.cuh",
+                  "rope_paged_kv_b200/csrc/common.cuh", "rope_paged_kv_b200/csrc/pipeline.cuh",
                   "rope_paged_kv_b200/csrc/device_utils.cuh"]
 PROFILE = "profiles/rope_split_store_paged_ragged_llama3_8b_prefill.md"
 
@@ -49,6 +50,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="llama3_8b_prefill",
+                    help="the named workload timed as the main line (default: the headline)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other entry points and the CPU baseline")
     return ap.parse_args()
@@ -186,14 +189,221 @@ def bytes_bshd(w) -> int:
 
 # ----------------------------------------------------------------------- our arm --
 
-def run_ours(args):
+WORKLOADS = {
+    "llama3_8b_prefill": "rope_split_store_paged_ragged",
+    "per_head_norm": "fused_qk_rmsnorm_rope_paged",
+    "dual_band_minimax": "fused_dual_qk_rmsnorm_rope_paged",
+    "radd_minimax": "kv_cache_radd",
+    "decode_bshd": "qk_rope_bshd_continuous",
+}
+
+
+class Case:
+    """One named workload staged on the device: `step()` is one call of its entry point
+    through the C ABI with the inputs resident in HBM; `e2e_step()` is the same call through
+    the Python binding with the step's inputs copied in from pinned host memory and its
+    result copied back."""
+
+
+def make_case(name, seed, dev):
     import ctypes
 
     import torch
-    import torch.distributed as dist
 
     import rope_paged_kv_b200 as rs
     import workloads as W
+
+    def d(t):
+        return t.to(dev)
+
+    def paged(kv, storage):
+        return rs.PagedCache(storage[kv.k_offset:],
+                             None if kv.v_offset is None else storage[kv.v_offset:],
+                             d(kv.page_table), d(kv.cache_lengths), kv.n_kv_heads,
+                             kv.head_dim, kv.page_size, kv.num_pages, kv.num_layers,
+                             kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride)
+
+    lib = rs.raw_library()
+    stream = torch.cuda.current_stream()
+    c = Case()
+    c.name, c.entry_point = name, WORKLOADS[name]
+    c.err = torch.zeros(1, dtype=torch.int32, device=dev)
+    keep = []
+
+    def bind(fn, args, where):
+        def step():
+            st = fn(*args)
+            if st != 0:
+                raise rs.RopeError(st, where)
+        return step
+
+    def pinned(t):
+        return t.contiguous().pin_memory()
+
+    if name in ("llama3_8b_prefill", "per_head_norm"):
+        w = W.llama3_8b_prefill(seed) if name == "llama3_8b_prefill" else W.per_head_norm(seed)
+        kv = w.cache
+        storage = d(kv.storage)
+        cache = paged(kv, storage)
+        qkv, offs, q_out = d(w.qkv), d(w.offsets), d(w.q_out)
+        fr = rs.Freqs(d(w.rope.table), w.rope.interleaved)
+        c_f, c_kv = fr.c(), cache.c()
+        keep += [c_f, c_kv]
+        if w.q_gamma is None:
+            args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
+                    offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), w.layer_idx,
+                    q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(), stream.cuda_stream)
+            c.step = bind(lib.rope_split_store_paged_ragged, args, c.entry_point)
+
+            def call():
+                rs.rope_split_store_paged_ragged(qkv, w.n_q_heads, offs, fr, cache, w.layer_idx,
+                                                 q_out, c.err)
+        else:
+            qg, kg = d(w.q_gamma), d(w.k_gamma)
+            args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
+                    offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), qg.data_ptr(),
+                    kg.data_ptr(), ctypes.c_float(w.epsilon), ctypes.c_float(w.weight_offset), 1,
+                    w.layer_idx, q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(),
+                    stream.cuda_stream)
+            c.step = bind(lib.fused_qk_rmsnorm_rope_paged, args, c.entry_point)
+
+            def call():
+                rs.fused_qk_rmsnorm_rope_paged(qkv, w.n_q_heads, offs, fr, cache, qg, kg,
+                                               w.epsilon, w.weight_offset, w.layer_idx, q_out,
+                                               True, c.err)
+        c.tokens = w.total_tokens
+        c.alg_bytes = bytes_ragged(w)
+        c.e2e_in = [(pinned(w.qkv), qkv), (pinned(w.offsets), offs),
+                    (pinned(kv.cache_lengths), cache.cache_lengths),
+                    (pinned(kv.page_table), cache.page_table)]
+        c.e2e_out = [(q_out, torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory())]
+        c.call = call
+        c.config = {"n_q_heads": w.n_q_heads, "n_kv_heads": kv.n_kv_heads,
+                    "head_dim": kv.head_dim, "page_size": kv.page_size,
+                    "batch": len(w.lengths), "lengths": w.lengths,
+                    "rope": f"{'interleaved' if w.rope.interleaved else 'half-split'}, "
+                            f"rope_dim {w.rope.rope_dim}, freqs_cis {w.rope.dtype}",
+                    "rmsnorm": w.q_gamma is not None}
+        c.workload = w
+    elif name == "dual_band_minimax":
+        w = W.dual_band_minimax(seed)
+        inp, offs = d(w.input), d(w.offsets)
+        ms, ist = d(w.main_cache.storage), d(w.index_cache.storage)
+        g = [d(x) for x in w.gammas]
+        qm, qi = d(w.q_main_out), d(w.q_index_out)
+        main = rs.NormBand(inp, *w.main_cols, w.main_q_heads, paged(w.main_cache, ms), g[0],
+                           g[1], w.main_eps, qm)
+        index = rs.NormBand(inp, *w.index_cols, w.index_q_heads, paged(w.index_cache, ist),
+                            g[2], g[3], w.index_eps, qi)
+        fr = rs.Freqs(d(w.rope.table), w.rope.interleaved)
+        mb, ib, c_f = main.c(keep), index.c(keep), fr.c()
+        keep += [mb, ib, c_f]
+        args = (ctypes.byref(mb), ctypes.byref(ib), offs.data_ptr(), offs.shape[0] - 1,
+                w.total_tokens, ctypes.byref(c_f), ctypes.c_float(w.weight_offset), 1,
+                w.layer_idx, c.err.data_ptr(), stream.cuda_stream)
+        c.step = bind(lib.fused_dual_qk_rmsnorm_rope_paged, args, c.entry_point)
+
+        def call():
+            rs.fused_dual_qk_rmsnorm_rope_paged(main, index, offs, w.total_tokens, fr,
+                                                w.weight_offset, w.layer_idx, True, c.err)
+        c.call = call
+        c.tokens = w.total_tokens
+        c.alg_bytes = bytes_dual(w)
+        c.e2e_in = [(pinned(w.input), inp), (pinned(w.offsets), offs),
+                    (pinned(w.main_cache.cache_lengths), main.cache.cache_lengths),
+                    (pinned(w.main_cache.page_table), main.cache.page_table),
+                    (pinned(w.index_cache.cache_lengths), index.cache.cache_lengths),
+                    (pinned(w.index_cache.page_table), index.cache.page_table)]
+        c.e2e_out = [(qm, torch.empty(qm.shape, dtype=qm.dtype).pin_memory()),
+                     (qi, torch.empty(qi.shape, dtype=qi.dtype).pin_memory())]
+        c.config = {"main_heads": [w.main_q_heads, w.main_cache.n_kv_heads],
+                    "index_heads": [w.index_q_heads, w.index_cache.n_kv_heads],
+                    "head_dim": w.main_cache.head_dim, "rope_dim": w.rope.rope_dim,
+                    "page_size": [w.main_cache.page_size, w.index_cache.page_size],
+                    "batch": len(w.lengths)}
+        c.workload = w
+    elif name == "radd_minimax":
+        w = W.radd_minimax(seed)
+        st_, a, offs = d(w.cache.storage), d(w.a), d(w.offsets)
+        cache = paged(w.cache, st_)
+        c_kv = cache.c()
+        keep.append(c_kv)
+        args = (a.data_ptr(), a.stride(0), a.shape[0], ctypes.byref(c_kv), offs.data_ptr(),
+                offs.shape[0] - 1, w.batch_offset, w.layer_idx, c.err.data_ptr(),
+                stream.cuda_stream)
+        c.step = bind(lib.kv_cache_radd, args, c.entry_point)
+
+        def call():
+            rs.kv_cache_radd(a, cache, offs, w.batch_offset, w.layer_idx, c.err)
+        c.call = call
+        c.tokens = w.a.shape[0]
+        c.alg_bytes = bytes_radd(w)
+        c.e2e_in = [(pinned(w.a), a), (pinned(w.offsets), offs),
+                    (pinned(w.cache.cache_lengths), cache.cache_lengths),
+                    (pinned(w.cache.page_table), cache.page_table)]
+        c.e2e_out = [(c.err, torch.empty(1, dtype=torch.int32).pin_memory())]
+        c.config = {"n_kv_heads": w.cache.n_kv_heads, "head_dim": w.cache.head_dim,
+                    "page_size": w.cache.page_size, "batch": len(w.lengths)}
+        c.workload = w
+    elif name == "decode_bshd":
+        w = W.decode_bshd(seed)
+        kv = w.cache
+        st_, out = d(kv.storage), d(w.output)
+        cc = rs.ContCache(st_, None, d(kv.lookup_table), d(kv.cache_lengths), kv.n_kv_heads,
+                          kv.head_dim, kv.num_slots, kv.num_layers, kv.max_seq_len,
+                          kv.slot_stride, kv.layer_stride, kv.pos_stride, kv.head_stride)
+        q, fr, vl = d(w.q_proj), rs.Freqs(d(w.rope.table), w.rope.interleaved), d(w.valid_lengths)
+        c_c, c_f = cc.c(), fr.c()
+        keep += [c_c, c_f]
+        B, S, H, D = w.q_proj.shape
+        args = (q.data_ptr(), B, S, H, D, ctypes.byref(c_c), ctypes.byref(c_f), w.layer_idx,
+                vl.data_ptr(), out.data_ptr(), c.err.data_ptr(), stream.cuda_stream)
+        c.step = bind(lib.qk_rope_bshd_continuous, args, c.entry_point)
+
+        def call():
+            rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl, out, c.err)
+        c.call = call
+        c.tokens = B * S
+        c.alg_bytes = bytes_bshd(w)
+        c.e2e_in = [(pinned(w.q_proj), q), (pinned(w.valid_lengths), vl),
+                    (pinned(kv.cache_lengths), cc.cache_lengths),
+                    (pinned(kv.lookup_table), cc.lookup_table)]
+        c.e2e_out = [(out, torch.empty(out.shape, dtype=out.dtype).pin_memory())]
+        c.config = {"q_proj": list(w.q_proj.shape), "n_kv_heads": kv.n_kv_heads,
+                    "cache": [kv.num_slots, kv.max_seq_len], "rope": "interleaved, freqs bf16"}
+        c.workload = w
+    else:
+        raise ValueError(name)
+    c.keep = keep
+    c.h2d = sum(h.numel() * h.element_size() for h, _ in c.e2e_in)
+    c.d2h = sum(h.numel() * h.element_size() for _, h in c.e2e_out)
+
+    def e2e_step():
+        for h, dv in c.e2e_in:
+            dv.copy_(h, non_blocking=True)
+        c.call()
+        for dv, h in c.e2e_out:
+            h.copy_(dv, non_blocking=True)
+    c.e2e_step = e2e_step
+    return c
+
+
+def time_steps(torch, step, flush, k, stream):
+    """Device time (ms) of k calls of step(), each after an L2 flush outside its events."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(k)]
+    for i in range(k):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -208,97 +418,40 @@ def run_ours(args):
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    def d(t):
-        return t.to(dev)
-
     # this rank's replica: its own seeded batch
-    w = W.llama3_8b_prefill(seed=1000 * rank)
-    kv = w.cache
-    storage = d(kv.storage)
-    cache = rs.PagedCache(storage[kv.k_offset:], storage[kv.v_offset:], d(kv.page_table),
-                          d(kv.cache_lengths), kv.n_kv_heads, kv.head_dim, kv.page_size,
-                          kv.num_pages, kv.num_layers, kv.page_stride, kv.layer_stride,
-                          kv.slot_stride, kv.head_stride)
-    qkv, offs, q_out = d(w.qkv), d(w.offsets), d(w.q_out)
-    freqs = rs.Freqs(d(w.rope.table), w.rope.interleaved)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    case = make_case(args.workload, 1000 * rank, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    # the C entry point with its arguments marshalled once
-    lib = rs.raw_library()
-    c_f, c_kv = freqs.c(), cache.c()
-    c_args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
-              offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), w.layer_idx,
-              q_out.data_ptr(), q_out.stride(0), err.data_ptr(), stream.cuda_stream)
-
-    def step():
-        st = lib.rope_split_store_paged_ragged(*c_args)
-        if st != 0:
-            raise rs.RopeError(st, "rope_split_store_paged_ragged")
-
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
 
-    for _ in range(max(3, args.warmup)):
+    W_ = max(3, args.warmup)
+    for _ in range(W_):
         flush.zero_()
-        step()
+        case.step()
     torch.cuda.synchronize()
-    assert int(err.item()) == 0, "device error bits set on the benchmark workload"
+    if args.workload != "radd_minimax":   # radd accumulates: its data stays valid anyway
+        assert int(case.err.item()) == 0, "device error bits set on the benchmark workload"
 
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     barrier()
     torch.cuda.synchronize()
     t0 = time.time()
-    for k in range(K):
-        flush.zero_()
-        ev[k][0].record(stream)
-        step()
-        ev[k][1].record(stream)
-    torch.cuda.synchronize()
+    dev_ms = time_steps(torch, case.step, flush, K, stream)
     t1 = time.time()
     barrier()
-    dev_ms = sum(a.elapsed_time(b) for a, b in ev)
-    launches = K
 
-    # end to end: pinned host inputs in, q_out back out, through the Python binding
-    qkv_h = w.qkv.pin_memory()
-    offs_h, cl_h, pt_h = (w.offsets.pin_memory(), kv.cache_lengths.pin_memory(),
-                          kv.page_table.pin_memory())
-    q_out_h = torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (qkv_h, offs_h, cl_h, pt_h))
-    d2h = q_out_h.numel() * q_out_h.element_size()
     K_e2e = max(1, min(K, 200))
-
-    def e2e_step():
-        qkv.copy_(qkv_h, non_blocking=True)
-        offs.copy_(offs_h, non_blocking=True)
-        cache.cache_lengths.copy_(cl_h, non_blocking=True)
-        cache.page_table.copy_(pt_h, non_blocking=True)
-        rs.rope_split_store_paged_ragged(qkv, w.n_q_heads, offs, freqs, cache, w.layer_idx,
-                                         q_out, err)
-        q_out_h.copy_(q_out, non_blocking=True)
-
     for _ in range(3):
-        e2e_step()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(K_e2e)]
+        case.e2e_step()
     barrier()
     torch.cuda.synchronize()
-    for k in range(K_e2e):
-        flush.zero_()
-        ev2[k][0].record(stream)
-        e2e_step()
-        ev2[k][1].record(stream)
-    torch.cuda.synchronize()
+    e2e_ms = time_steps(torch, case.e2e_step, flush, K_e2e, stream)
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
     sampler.stop()
 
-    tokens = torch.tensor([float(w.total_tokens)], device=dev, dtype=torch.float64)
+    tokens = torch.tensor([float(case.tokens)], device=dev, dtype=torch.float64)
     times = torch.tensor([dev_ms, e2e_ms], device=dev, dtype=torch.float64)
     if world > 1:
         dist.all_reduce(tokens, op=dist.ReduceOp.SUM)
@@ -306,52 +459,42 @@ def run_ours(args):
     tok_all = float(tokens.item())
     dev_ms_max, e2e_ms_max = (float(x) for x in times.tolist())
 
-    extras = {}
-    cpu = None
+    peak, peak_src = measured_peak()
+    extras, cpu = {}, None
     if rank == 0 and world == 1 and not args.no_extras:
-        extras = run_entry_points(rs, W, dev, flush)
-        extras["rope_split_store_paged_ragged"] = {
-            "workload": w.name, "tokens": w.total_tokens,
-            "us_per_launch": round(dev_ms / K * 1e3, 2),
-            "tokens_per_s": round(w.total_tokens * K / (dev_ms / 1e3), 1),
-            "algorithmic_gbs": round(bytes_ragged(w) * K / (dev_ms / 1e3) / 1e9, 1)}
-        cpu = cpu_baseline(W)
+        extras = run_entry_points(torch, dev, flush, stream, args.workload, peak)
+        extras[args.workload] = summarize(case, dev_ms / K / 1e3, peak)
+        cpu = cpu_baseline(args.workload)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return
 
-    peak, peak_src = measured_peak()
-    alg = bytes_ragged(w)
     mean_s = dev_ms / K / 1e3
-    achieved = alg / mean_s / 1e9
-    for v in extras.values():
-        if "algorithmic_gbs" in v:
-            v["frac_of_measured_hbm"] = round(v["algorithmic_gbs"] / peak, 3)
+    achieved = case.alg_bytes / mean_s / 1e9
     line = {
         "metric": METRIC, "value": round(tok_all * K / (dev_ms_max / 1e3), 1), "unit": UNIT,
-        "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+        "n_gpus": world, "steps": K, "warmup": W_,
         "ms_per_step": round(dev_ms_max / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; shapes of a Llama-3-8B ragged prefill)",
-        "config": {"workload": w.name, "entry_point": "rope_split_store_paged_ragged",
-                   "tokens_per_rank": w.total_tokens, "batch": len(w.lengths),
-                   "lengths": w.lengths, "n_q_heads": w.n_q_heads,
-                   "n_kv_heads": kv.n_kv_heads, "head_dim": kv.head_dim,
-                   "page_size": kv.page_size, "rope": "half-split, rope_dim 128, theta 5e5, "
-                   "freqs_cis f32 [8192, 128]", "cache_dtype": "bf16",
-                   "l2": "flushed before every step (256 MiB memset outside the timed events)",
-                   "parallelism": f"replicas x{world} (each rank its own batch, no collective)"},
-        "gpu_launches": launches,
+        "data": "synthetic (seeded, shapes of the named workload)",
+        "config": dict({"workload": case.workload.name, "entry_point": case.entry_point,
+                        "tokens_per_rank": case.tokens, "cache_dtype": "bf16",
+                        "l2": "flushed before every step (256 MiB memset outside the timed "
+                              "events)",
+                        "parallelism": f"replicas x{world} (each rank its own batch, "
+                                       f"no collective)"}, **case.config),
+        "gpu_launches": K,
         "e2e": {"value": round(tok_all * K_e2e / (e2e_ms_max / 1e3), 1), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "path": "pinned host qkv/offsets/cache_lengths/page_table -> device, "
-                        "rope_paged_kv_b200.rope_split_store_paged_ragged, q_out -> pinned host"},
+                "h2d_bytes_per_step": case.h2d, "d2h_bytes_per_step": case.d2h,
+                "path": "pinned host inputs -> device copies, the rope_paged_kv_b200 call, "
+                        "the result -> pinned host, all inside the timed events"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(), "peak_source": peak_src,
-                     "algorithmic_bytes_per_launch": alg,
-                     "kernel": "banded_store_kernel<bf16, 128, store>"},
+                     "traffic": profiled_traffic() if args.workload == "llama3_8b_prefill"
+                     else None,
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": case.alg_bytes,
+                     "kernel": KERNELS[args.workload]},
         "clocks": sampler.summary(t0, t1),
     }
     if cpu is not None:
@@ -361,108 +504,55 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
-def time_launches(torch, launch, flush, reps=20, warm=3):
-    stream = torch.cuda.current_stream()
-    for _ in range(warm):
-        flush.zero_()
-        launch()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(reps)]
-    torch.cuda.synchronize()
-    for a, b in ev:
-        flush.zero_()
-        a.record(stream)
-        launch()
-        b.record(stream)
-    torch.cuda.synchronize()
-    return sum(a.elapsed_time(b) for a, b in ev) / reps / 1e3  # seconds per launch
+KERNELS = {"llama3_8b_prefill": "banded_store_kernel<bf16, head_dim 128, no norm>",
+           "per_head_norm": "banded_store_kernel<bf16, head_dim 128, rmsnorm>",
+           "dual_band_minimax": "banded_store_kernel<bf16, head_dim 128, rmsnorm> (two bands)",
+           "radd_minimax": "radd_kernel<bf16, head_dim 128>",
+           "decode_bshd": "bshd_rope_kernel<bf16, head_dim 128>"}
 
 
-def run_entry_points(rs, W, dev, flush):
-    """The other entry points on their named workloads (N=1 only; reported, not headline)."""
-    import torch
+def summarize(case, sec, peak):
+    gbs = case.alg_bytes / sec / 1e9
+    return {"workload": case.workload.name, "entry_point": case.entry_point,
+            "tokens": case.tokens, "us_per_launch": round(sec * 1e6, 2),
+            "tokens_per_s": round(case.tokens / sec, 1), "algorithmic_gbs": round(gbs, 1),
+            "frac_of_measured_hbm": round(gbs / peak, 3)}
 
-    def d(t):
-        return t.to(dev)
 
-    def paged(kv, storage):
-        return rs.PagedCache(storage[kv.k_offset:],
-                             None if kv.v_offset is None else storage[kv.v_offset:],
-                             d(kv.page_table), d(kv.cache_lengths), kv.n_kv_heads,
-                             kv.head_dim, kv.page_size, kv.num_pages, kv.num_layers,
-                             kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride)
-
+def run_entry_points(torch, dev, flush, stream, headline, peak, reps=20):
+    """Every other named workload, timed the same way (N=1 only; reported beside the
+    headline, not instead of it)."""
     out = {}
-
-    def record(name, w, tokens, nbytes, sec):
-        out[name] = {"workload": w.name, "tokens": tokens, "us_per_launch": round(sec * 1e6, 2),
-                     "tokens_per_s": round(tokens / sec, 1),
-                     "algorithmic_gbs": round(nbytes / sec / 1e9, 1)}
-
-    w = W.per_head_norm()
-    st, qo = d(w.cache.storage), d(w.q_out)
-    args = (d(w.qkv), w.n_q_heads, d(w.offsets), rs.Freqs(d(w.rope.table), w.rope.interleaved),
-            paged(w.cache, st), d(w.q_gamma), d(w.k_gamma), w.epsilon, w.weight_offset,
-            w.layer_idx, qo)
-    sec = time_launches(torch, lambda: rs.fused_qk_rmsnorm_rope_paged(*args), flush)
-    record("fused_qk_rmsnorm_rope_paged", w, w.total_tokens, bytes_ragged(w), sec)
-    del st, qo, args
-
-    w = W.dual_band_minimax()
-    inp = d(w.input)
-    ms, ist = d(w.main_cache.storage), d(w.index_cache.storage)
-    g = [d(x) for x in w.gammas]
-    main = rs.NormBand(inp, *w.main_cols, w.main_q_heads, paged(w.main_cache, ms), g[0], g[1],
-                       w.main_eps, d(w.q_main_out))
-    index = rs.NormBand(inp, *w.index_cols, w.index_q_heads, paged(w.index_cache, ist), g[2],
-                        g[3], w.index_eps, d(w.q_index_out))
-    offs, fr = d(w.offsets), rs.Freqs(d(w.rope.table), w.rope.interleaved)
-    sec = time_launches(torch, lambda: rs.fused_dual_qk_rmsnorm_rope_paged(
-        main, index, offs, w.total_tokens, fr, w.weight_offset, w.layer_idx), flush)
-    record("fused_dual_qk_rmsnorm_rope_paged", w, w.total_tokens, bytes_dual(w), sec)
-    del inp, ms, ist, main, index
-
-    w = W.radd_minimax()
-    st = d(w.cache.storage)
-    a, offs, kvr = d(w.a), d(w.offsets), None
-    kvr = paged(w.cache, st)
-    sec = time_launches(torch, lambda: rs.kv_cache_radd(a, kvr, offs, w.batch_offset,
-                                                        w.layer_idx), flush)
-    record("kv_cache_radd", w, w.a.shape[0], bytes_radd(w), sec)
-    del st, a, kvr
-
-    w = W.decode_bshd()
-    st, out_t = d(w.cache.storage), d(w.output)
-    kv = w.cache
-    cc = rs.ContCache(st, None, d(kv.lookup_table), d(kv.cache_lengths), kv.n_kv_heads,
-                      kv.head_dim, kv.num_slots, kv.num_layers, kv.max_seq_len, kv.slot_stride,
-                      kv.layer_stride, kv.pos_stride, kv.head_stride)
-    q, fr, vl = d(w.q_proj), rs.Freqs(d(w.rope.table), w.rope.interleaved), d(w.valid_lengths)
-    sec = time_launches(torch, lambda: rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl,
-                                                                  out_t), flush)
-    B, S = w.q_proj.shape[:2]
-    record("qk_rope_bshd_continuous", w, B * S, bytes_bshd(w), sec)
-    # back-to-back launches without the flush (the decode step's L2-warm case)
-    stream = torch.cuda.current_stream()
-    a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(3):
-        rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl, out_t)
-    a0.record(stream)
-    n = 50
-    for _ in range(n):
-        rs.qk_rope_bshd_continuous(q, cc, fr, w.layer_idx, vl, out_t)
-    b0.record(stream)
-    torch.cuda.synchronize()
-    out["qk_rope_bshd_continuous"]["us_per_launch_back_to_back_l2_warm"] = round(
-        a0.elapsed_time(b0) / n * 1e3, 2)
-    del st, out_t, cc, q
-    torch.cuda.empty_cache()
+    for name in WORKLOADS:
+        if name == headline:
+            continue
+        case = make_case(name, 0, dev)
+        for _ in range(3):
+            flush.zero_()
+            case.step()
+        sec = time_steps(torch, case.step, flush, reps, stream) / reps / 1e3
+        out[name] = summarize(case, sec, peak)
+        if name == "decode_bshd":
+            # back-to-back launches without the flush (the decode step's L2-warm case)
+            a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(50):
+                case.step()
+            b0.record(stream)
+            torch.cuda.synchronize()
+            out[name]["us_per_launch_back_to_back_l2_warm"] = round(a0.elapsed_time(b0) / 50 * 1e3, 2)
+        del case
+        torch.cuda.empty_cache()
     return out
 
 
-def cpu_baseline(W, min_seconds=10.0, max_reps=20):
-    """The oracle as it stands (single-threaded C, double precision) on the same workload."""
+def cpu_baseline(workload, min_seconds=10.0, max_reps=20):
+    """The oracle as it stands (single-threaded C, double precision) on the headline
+    workload's batch (the same seeded batch rank 0 measured)."""
+    import workloads as W
     from oracle import runners as R
+    if workload != "llama3_8b_prefill":
+        return None
     w = W.llama3_8b_prefill(seed=0)
     reps, t_total = 0, 0.0
     while t_total < min_seconds and reps < max_reps:

@@ -62,6 +62,7 @@ typedef enum { ROPE_DTYPE_BF16 = 0, ROPE_DTYPE_F16 = 1, ROPE_DTYPE_F32 = 2 } rop
 #define ROPE_DEVERR_PAGE_INDEX 0x4u  /* position / page_size >= max_pages_per_seq */
 #define ROPE_DEVERR_PAGE_ID 0x8u     /* page-table entry >= num_pages */
 #define ROPE_DEVERR_BATCH 0x10u      /* sequence (+ batch_offset) >= n_seqs, or slot >= num_slots */
+#define ROPE_DEVERR_TIMEOUT 0x20u    /* an internal pipeline wait gave up (the call is incomplete) */
 
 /* freqs_cis [max_seq_len, rope_dim], row-major, contiguous.  Row p holds rope_dim/2
  * pairs (cos, sin): column 2i is cos and 2i+1 is sin of pair i's angle at position p (the
@@ -76,7 +77,8 @@ typedef enum { ROPE_DTYPE_BF16 = 0, ROPE_DTYPE_F16 = 1, ROPE_DTYPE_F32 = 2 } rop
  * o = rope_col_offset, or head_dim - rope_dim when rope_col_offset < 0: partial RoPE
  * rotates the last rope_dim columns of each head unless the caller says otherwise.
  * Supported: o and rope_dim multiples of the 16-byte vector width (8 elements for 16-bit
- * types, 4 for F32), and for the half-split layout rope_dim/2 too. */
+ * types, 4 for F32), and for the half-split layout rope_dim/2 too; a table row
+ * (rope_dim * element size) is a multiple of 16 bytes and the table is 16-byte aligned. */
 typedef struct {
   const void *data;
   int32_t dtype; /* rope_dtype_t of the table */

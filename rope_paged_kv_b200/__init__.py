@@ -35,7 +35,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "rope_store.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA = 0, 1, 2, 3
 DEVERR_ROW_OFFSETS, DEVERR_POSITION, DEVERR_PAGE_INDEX = 0x1, 0x2, 0x4
-DEVERR_PAGE_ID, DEVERR_BATCH = 0x8, 0x10
+DEVERR_PAGE_ID, DEVERR_BATCH, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
 
 _DTYPE_CODE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 

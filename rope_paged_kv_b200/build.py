@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librope_store.so")
 SOURCES = [os.path.join(CSRC, "rope_store.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "device_utils.cuh"),
+HEADERS = ["device_utils.cuh", "pipeline.cuh", "common.cuh", "banded.cuh", "bshd.cuh", "radd.cuh"]
+DEPS = SOURCES + [os.path.join(CSRC, h) for h in HEADERS] + [
                   os.path.join(ROOT, "include", "rope_store.h")]
 
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
