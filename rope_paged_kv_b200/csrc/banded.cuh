@@ -24,9 +24,12 @@
 
 namespace rs {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumers = 32 * kConsumerWarps;
-constexpr int kPipeThreads = kConsumers + 64;  // + producer warp + storer warp
+// A CTA is a producer warp, a storer warp and CW consumer warps; the storer keeps LAG
+// bulk-store groups in flight before handing a stage back.  Two shapes are built: a light
+// one (4 consumer warps, more CTAs per SM) for little work per token, and a heavy one
+// (8 consumer warps) for RMSNorm and many heads.
+template <int CW>
+__host__ __device__ constexpr int pipe_threads() { return 32 * (CW + 2); }
 
 struct BandDev {
   const void *input;
@@ -112,12 +115,95 @@ __device__ __forceinline__ void load_lane_freqs(const void *F, int fdt, bool int
   }
 }
 
-template <typename T, int D, bool NORM>
-__global__ void __launch_bounds__(kPipeThreads, 2)
+// Load C consecutive 16-byte chunks at `p` (shared memory) into out[0..C).  The lanes of a
+// head-row group read neighbouring C*16-byte runs; issuing chunk (k + rot) % C at step k,
+// with rot = (lane-in-group / lanes-per-128B) % C, puts the 8 lanes of a quarter-warp on 8
+// different 16-byte bank groups.  The rotation is undone with fixed selects.
+template <int C>
+__device__ __forceinline__ void lds_chunks(const unsigned char *p, int rot, uint4 (&out)[C]) {
+  uint4 t[C];
+#pragma unroll
+  for (int k = 0; k < C; ++k) t[k] = ld_shared_v4(p + ((k + rot) % C) * 16);
+  // t[k] holds chunk (k + rot) % C: rotate right by rot
+#pragma unroll
+  for (int k = 0; k < C; ++k) out[k] = t[k];
+  if constexpr (C >= 2) {
+    if (rot & 1) {
+#pragma unroll
+      for (int k = 0; k < C; ++k) out[(k + 1) % C] = t[k];
+#pragma unroll
+      for (int k = 0; k < C; ++k) t[k] = out[k];
+    }
+  }
+  if constexpr (C >= 4) {
+    if (rot & 2) {
+#pragma unroll
+      for (int k = 0; k < C; ++k) out[(k + 2) % C] = t[k];
+    }
+  }
+}
+
+// M consecutive table values (element type fdt) starting at element `col` of the shared
+// row F, widened to float, read bank-conflict free across the lanes of a group (`gl` =
+// lane index inside the group).
+template <int M>
+__device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int col, int gl,
+                                          float (&f)[M]) {
+  if (fdt == 2) {
+    constexpr int C = M / 4;           // 16-byte chunks per lane
+    constexpr int LP = 32 / M > 0 ? 32 / M : 1;  // lanes sharing one 128-byte line
+    uint4 c[C];
+    lds_chunks<C>(F + col * 4, (gl / LP) % C, c);
+#pragma unroll
+    for (int k = 0; k < C; ++k) {
+      f[4 * k] = __uint_as_float(c[k].x);
+      f[4 * k + 1] = __uint_as_float(c[k].y);
+      f[4 * k + 2] = __uint_as_float(c[k].z);
+      f[4 * k + 3] = __uint_as_float(c[k].w);
+    }
+  } else {
+    constexpr int C = M / 8 > 0 ? M / 8 : 1;
+    uint32_t w[C * 4];
+    if constexpr (M >= 8) {
+      constexpr int LP = 64 / M;
+      uint4 c[C];
+      lds_chunks<C>(F + col * 2, (gl / LP) % C, c);
+#pragma unroll
+      for (int k = 0; k < C; ++k) {
+        w[4 * k] = c[k].x;
+        w[4 * k + 1] = c[k].y;
+        w[4 * k + 2] = c[k].z;
+        w[4 * k + 3] = c[k].w;
+      }
+    } else {
+      const uint2 v = *reinterpret_cast<const uint2 *>(F + col * 2);
+      w[0] = v.x;
+      w[1] = v.y;
+    }
+#pragma unroll
+    for (int i = 0; i < M / 2; ++i) {
+      const unsigned short lo = (unsigned short)(w[i] & 0xffffu), hi = (unsigned short)(w[i] >> 16);
+      if (fdt == 0) {
+        f[2 * i] = __uint_as_float((uint32_t)lo << 16);
+        f[2 * i + 1] = __uint_as_float((uint32_t)hi << 16);
+      } else {
+        f[2 * i] = __half2float(__ushort_as_half(lo));
+        f[2 * i + 1] = __half2float(__ushort_as_half(hi));
+      }
+    }
+  }
+}
+
+template <typename T, int D, bool NORM, int CW, int LAG>
+__global__ void __launch_bounds__(pipe_threads<CW>(), 2)
     banded_store_kernel(const __grid_constant__ BandedParams p) {
+  constexpr int kConsumerWarps = CW;
+  constexpr int kConsumers = 32 * CW;
+  constexpr int kPipeThreads = pipe_threads<CW>();
+  constexpr int kStoreLag = LAG;
   using VT = Vec<T>;
   constexpr int N = VT::N;
-  constexpr int L = D / N;                 // lanes per head row
+  constexpr int L = D / (2 * N);           // lanes per head row: each lane owns 2 vectors
   constexpr int G = kConsumers / L;        // head rows per consumer pass
   constexpr int EB = (int)sizeof(T);
   static_assert(L <= 32 && 32 % L == 0, "a head row must fit in one warp");
@@ -285,28 +371,54 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           }
         }
         bulk_commit();
-        bulk_wait_read<0>();
-        mbar_arrive(&empty[s]);
+        // hand back the stage whose stores were issued kStoreLag tokens ago once they have
+        // read it; up to kStoreLag newer groups may still be reading
+        if (i >= kStoreLag) {
+          bulk_wait_read<kStoreLag>();
+          mbar_arrive(&empty[(i - kStoreLag) % p.S]);
+        }
       }
+      bulk_wait_read<0>();
+      for (int i = max(0, n_local - kStoreLag); i < n_local; ++i) mbar_arrive(&empty[i % p.S]);
       bulk_wait<0>();
     }
   } else {
     // ------------------------------------------------------------------ consumers --
+    // A head row is D / N 16-byte vectors; lane j of its group of L lanes owns two of them,
+    // va and vb.  Half-split: the first R/(2N) lanes own a rotation pair each (vector
+    // o/N + j and its partner R/(2N) vectors later), the other lanes own two unrotated
+    // vectors.  Interleaved: lane j owns vectors j and j + L.
     const int ctid = tid - 64;
     const int li = ctid % L, grp = ctid / L;
-    const int c0 = li * N;
     const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
     const RopeDev &rp = p.rope;
-    const bool in_rope = lane_in_rope(rp, c0);
     const bool inter = rp.interleaved != 0;
-    const int half = rp.R >> 1;
-    const bool first = !inter && in_rope && (c0 - rp.off) < half;
-    // element distance to the half-split partner vector, and this lane's first table column
-    const int pdelta = (inter || !in_rope) ? 0 : (first ? half : -half);
-    const int fcol = inter ? (c0 - rp.off) : 2 * (first ? (c0 - rp.off) : (c0 - rp.off - half));
-    const bool busy = NORM || in_rope;  // lanes with nothing to do leave their bytes in place
-    // the lanes of this group that write back (partners must have read first)
-    const unsigned smask = gmask & __ballot_sync(0xffffffffu, busy);
+    const int ov = rp.off / N, rv = rp.R / N;  // first rotated vector, rotated vectors
+    int va, vb;
+    bool rot_a, rot_b;
+    if (inter) {
+      va = li;
+      vb = li + L;
+      rot_a = va >= ov && va < ov + rv;
+      rot_b = vb >= ov && vb < ov + rv;
+    } else if (li < rv / 2) {
+      va = ov + li;
+      vb = ov + li + rv / 2;
+      rot_a = rot_b = true;
+    } else {
+      // the k-th unrotated vector, k < (D/N - rv) / 2, and the one half of those later
+      const int k = li - rv / 2, np = D / N - rv;
+      const int ka = k, kb = k + np / 2;
+      va = ka < ov ? ka : ka + rv;
+      vb = kb < ov ? kb : kb + rv;
+      rot_a = rot_b = false;
+    }
+    const bool busy = NORM || rot_a || rot_b;  // lanes with nothing to do leave bytes in place
+    const int ca = va * N, cb = vb * N;         // first columns of the two vectors
+    // table columns: interleaved, vector v uses F[v*N - off ..]; half-split pair uses
+    // F[2 * (ca - off) ..] (cos, sin of pair ca - off + e)
+    const int fa = inter ? ca - rp.off : 2 * (ca - rp.off);
+    const int fb = cb - rp.off;
     // this thread's head rows of a token, decoded once into shared memory
     const int n_items = (p.work_total + G - 1) / G;
     uint32_t *item = s_items + ctid;  // slot u at item[u * kConsumers]
@@ -318,13 +430,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         const BandDev &bd = band ? p.band[1] : p.band[0];
         const int r = j - (band ? p.work0 : 0);  // Q heads then K heads: stage rows 0..
         const int kind = r >= bd.n_q ? 1 : 0;
-        const uint32_t soff = (uint32_t)(bd.smem_off + (r * D + c0) * EB);
+        const uint32_t soff = (uint32_t)(bd.smem_off + r * D * EB);
         w = kItemAct | (uint32_t)band << kItemBandShift | (uint32_t)kind << kItemKindShift | soff;
       }
       item[u * kConsumers] = w;
     }
-    float fc[N], fs[N];  // this token's (cos, sin) for this lane, current band
-    float g[N], gp[N];   // gamma + weight_offset of this lane's and its partner's columns
+    // per token: (cos, sin) of this lane's columns; per (band, kind): gamma + weight_offset
+    float fca[N], fsa[N], fcb[N], fsb[N];
+    float ga[N], gb[N];
+    int g_sel = -1;
     for (int i = 0; i < n_local; ++i) {
       const int s = i % p.S;
       if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
@@ -336,7 +450,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
       }
       unsigned char *st = stages + (size_t)s * p.stage_bytes;
       const int ok0 = meta[s].ok[0], ok1 = meta[s].ok[1];
-      int f_band = -1, g_sel = -1;
+      int f_band = -1;
 #pragma unroll 1
       for (int u = 0; u < n_items; ++u) {
         const uint32_t w = item[u * kConsumers];
@@ -344,87 +458,101 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         const int band = (w >> kItemBandShift) & 1;
         if (!(band ? ok1 : ok0)) continue;
         const int kind = (w >> kItemKindShift) & 1;
-        unsigned char *src = st + (w & kItemOffMask);
-        float x[N], xp[N];
-        VT::widen(ld_shared_v4(src), x);
-        const bool pair_lane = pdelta != 0;
-        if (pair_lane) VT::widen(ld_shared_v4(src + pdelta * EB), xp);
-        if constexpr (NORM) {
-          if (g_sel != band * 2 + kind) {
-            g_sel = band * 2 + kind;
-            const float4 *gr = reinterpret_cast<const float4 *>(s_gamma + g_sel * D + c0);
+        const BandDev &bd = band ? p.band[1] : p.band[0];
+        if ((rot_a || rot_b) && f_band != band) {  // this token's table row for the band
+          f_band = band;
+          const unsigned char *F = st + bd.f_off;
+          if (inter) {
+            float f[N];
+            if (rot_a) {
+              lds_freqs<N>(F, rp.dtype, fa, li, f);
 #pragma unroll
-            for (int e = 0; e < N / 4; ++e) {
-              const float4 v = gr[e];
-              g[4 * e] = v.x;
-              g[4 * e + 1] = v.y;
-              g[4 * e + 2] = v.z;
-              g[4 * e + 3] = v.w;
-            }
-            if (pair_lane) {
-              const float4 *gq = reinterpret_cast<const float4 *>(s_gamma + g_sel * D + c0 + pdelta);
-#pragma unroll
-              for (int e = 0; e < N / 4; ++e) {
-                const float4 v = gq[e];
-                gp[4 * e] = v.x;
-                gp[4 * e + 1] = v.y;
-                gp[4 * e + 2] = v.z;
-                gp[4 * e + 3] = v.w;
+              for (int e = 0; e < N; e += 2) {
+                fca[e] = fca[e + 1] = f[e];
+                fsa[e] = fsa[e + 1] = f[e + 1];
               }
             }
+            if (rot_b) {
+              lds_freqs<N>(F, rp.dtype, fb, li, f);
+#pragma unroll
+              for (int e = 0; e < N; e += 2) {
+                fcb[e] = fcb[e + 1] = f[e];
+                fsb[e] = fsb[e + 1] = f[e + 1];
+              }
+            }
+          } else {
+            float f[2 * N];
+            lds_freqs<2 * N>(F, rp.dtype, fa, li, f);
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+              fca[e] = f[2 * e];
+              fsa[e] = f[2 * e + 1];
+            }
           }
-          const BandDev &bd = band ? p.band[1] : p.band[0];
+        }
+        unsigned char *row = st + (w & kItemOffMask);
+        float xa[N], xb[N];
+        VT::widen(ld_shared_v4(row + ca * EB), xa);
+        VT::widen(ld_shared_v4(row + cb * EB), xb);
+        if constexpr (NORM) {
+          if (g_sel != band * 2 + kind) {  // gamma does not depend on the token: kept
+            g_sel = band * 2 + kind;
+            const unsigned char *gr = reinterpret_cast<const unsigned char *>(s_gamma + g_sel * D);
+            lds_freqs<N>(gr, 2, ca, li, ga);
+            lds_freqs<N>(gr, 2, cb, li, gb);
+          }
           float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int e = 0; e < N; e += 2)
-            acc = __ffma2_rn(make_float2(x[e], x[e + 1]), make_float2(x[e], x[e + 1]), acc);
+          for (int e = 0; e < N; e += 2) {
+            acc = __ffma2_rn(make_float2(xa[e], xa[e + 1]), make_float2(xa[e], xa[e + 1]), acc);
+            acc = __ffma2_rn(make_float2(xb[e], xb[e + 1]), make_float2(xb[e], xb[e + 1]), acc);
+          }
           float ss = acc.x + acc.y;
 #pragma unroll
           for (int msk = L / 2; msk > 0; msk >>= 1) ss += __shfl_xor_sync(gmask, ss, msk);
           const float r = rsqrtf(ss * (1.0f / D) + bd.eps);
+          const float2 rr = make_float2(r, r);
 #pragma unroll
           for (int e = 0; e < N; e += 2) {
-            const float2 rg = __fmul2_rn(make_float2(r, r), make_float2(g[e], g[e + 1]));
-            const float2 y = __fmul2_rn(make_float2(x[e], x[e + 1]), rg);
-            x[e] = y.x;
-            x[e + 1] = y.y;
-          }
-          if (pair_lane) {
-#pragma unroll
-            for (int e = 0; e < N; e += 2) {
-              const float2 rg = __fmul2_rn(make_float2(r, r), make_float2(gp[e], gp[e + 1]));
-              const float2 y = __fmul2_rn(make_float2(xp[e], xp[e + 1]), rg);
-              xp[e] = y.x;
-              xp[e + 1] = y.y;
-            }
+            const float2 ya = __fmul2_rn(make_float2(xa[e], xa[e + 1]),
+                                         __fmul2_rn(rr, make_float2(ga[e], ga[e + 1])));
+            const float2 yb = __fmul2_rn(make_float2(xb[e], xb[e + 1]),
+                                         __fmul2_rn(rr, make_float2(gb[e], gb[e + 1])));
+            xa[e] = ya.x; xa[e + 1] = ya.y;
+            xb[e] = yb.x; xb[e + 1] = yb.y;
           }
         }
-        if (in_rope) {
-          if (f_band != band) {
-            f_band = band;
-            load_lane_freqs<N>(st + (band ? p.band[1] : p.band[0]).f_off, rp.dtype, inter, first,
-                               fcol, fc, fs);
+        if (inter) {
+          if (rot_a) {
+#pragma unroll
+            for (int e = 0; e < N; e += 2) {
+              const float a = xa[e], b = xa[e + 1];
+              xa[e] = fmaf(a, fca[e], -b * fsa[e]);
+              xa[e + 1] = fmaf(a, fsa[e], b * fca[e]);
+            }
           }
-          if (inter) {
+          if (rot_b) {
 #pragma unroll
             for (int e = 0; e < N; e += 2) {
-              const float a = x[e], b = x[e + 1];
-              x[e] = fmaf(a, fc[e], -b * fs[e]);
-              x[e + 1] = fmaf(a, fs[e], b * fc[e]);
+              const float a = xb[e], b = xb[e + 1];
+              xb[e] = fmaf(a, fcb[e], -b * fsb[e]);
+              xb[e + 1] = fmaf(a, fsb[e], b * fcb[e]);
             }
-          } else {
+          }
+        } else if (rot_a) {
+          // (a, b) -> (a c - b s, a s + b c), pair e of vector va with pair e of vector vb
 #pragma unroll
-            for (int e = 0; e < N; e += 2) {
-              const float2 y = __ffma2_rn(make_float2(xp[e], xp[e + 1]), make_float2(fs[e], fs[e + 1]),
-                                          __fmul2_rn(make_float2(x[e], x[e + 1]),
-                                                     make_float2(fc[e], fc[e + 1])));
-              x[e] = y.x;
-              x[e + 1] = y.y;
-            }
+          for (int e = 0; e < N; e += 2) {
+            const float2 a = make_float2(xa[e], xa[e + 1]), b = make_float2(xb[e], xb[e + 1]);
+            const float2 c = make_float2(fca[e], fca[e + 1]), sn = make_float2(fsa[e], fsa[e + 1]);
+            const float2 ya = __ffma2_rn(b, make_float2(-sn.x, -sn.y), __fmul2_rn(a, c));
+            const float2 yb = __ffma2_rn(a, sn, __fmul2_rn(b, c));
+            xa[e] = ya.x; xa[e + 1] = ya.y;
+            xb[e] = yb.x; xb[e + 1] = yb.y;
           }
         }
-        if (!inter) __syncwarp(smask);  // partners have read before anyone writes back
-        st_shared_v4(src, VT::narrow(x));
+        if (NORM || rot_a) st_shared_v4(row + ca * EB, VT::narrow(xa));
+        if (NORM || rot_b) st_shared_v4(row + cb * EB, VT::narrow(xb));
       }
       fence_proxy_async_smem();  // the storer's bulk copies read what was written here
       __syncwarp();

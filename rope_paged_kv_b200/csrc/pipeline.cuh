@@ -13,6 +13,9 @@
 
 namespace rs {
 
+#ifndef ROPE_WAIT_BACKOFF_NS
+#define ROPE_WAIT_BACKOFF_NS 32
+#endif
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // a wait longer than 2 s counts as stuck
 constexpr uint32_t kSpinLimit = 1u << 30;          // and so does this many polls
 
@@ -66,6 +69,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   uint64_t t0 = 0;
   for (uint32_t it = 0; it < kSpinLimit; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+#if ROPE_WAIT_BACKOFF_NS > 0
+    if (it >= 2) __nanosleep(ROPE_WAIT_BACKOFF_NS);  // leave the issue slots to busy warps
+#endif
     if ((it & 63u) == 63u) {
       if (*abort) return false;
       const uint64_t now = global_ns();

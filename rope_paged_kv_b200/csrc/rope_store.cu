@@ -18,8 +18,19 @@
 namespace rs {
 
 constexpr int kSmemSeqs = 1024;         // batches up to this size stage offsets in smem
-constexpr int kStageTarget = 96 << 10;  // shared memory given to the stage ring per CTA
 constexpr int kMaxStages = 8;
+
+// Launch shapes of the banded kernel (measured on B200 over the named workloads): consumer
+// warps, store lag and the shared memory given to a CTA's stage ring.
+struct BandedShape {
+  int cw, lag, ring_kb;
+};
+constexpr BandedShape kLightShape = {4, 2, 64};  // <= 64 head rows of Q+K per token, no norm
+constexpr BandedShape kHeavyShape = {8, 0, 96};  // RMSNorm or many heads
+
+static BandedShape pick_shape(const BandedParams &p, bool norm) {
+  return (!norm && p.work_total <= 64) ? kLightShape : kHeavyShape;
+}
 
 // ------------------------------------------------------------------------ host side --
 
@@ -207,7 +218,8 @@ static int elem_bytes_of(const BandedParams &p) { return p.elem_bytes; }
 
 // Shared-memory layout of the banded kernel: [stages | full, empty barriers | metadata |
 // gammas | offsets, cache lengths].  Returns the dynamic shared memory size.
-static size_t layout_banded(BandedParams &p, int D, bool norm) {
+static size_t layout_banded(BandedParams &p, int D, bool norm, const BandedShape &sh) {
+  const int kConsumers = 32 * sh.cw, kStoreLag = sh.lag, kStageTarget = sh.ring_kb << 10;
   int64_t off = 0;
   for (int k = 0; k < p.n_bands; ++k) {
     BandDev &bd = p.band[k];
@@ -222,7 +234,9 @@ static size_t layout_banded(BandedParams &p, int D, bool norm) {
   }
   p.stage_bytes = (int32_t)round_up(off, 128);
   int S = (int)(kStageTarget / p.stage_bytes);
-  S = S < 2 ? 2 : (S > kMaxStages ? kMaxStages : S);
+  // the storer holds up to kStoreLag + 1 stages; keep at least two for loading / compute
+  S = S < kStoreLag + 3 ? kStoreLag + 3 : (S > kMaxStages ? kMaxStages : S);
+  if (S < 3) S = 3;
   p.S = S;
   int64_t total = (int64_t)S * p.stage_bytes;
   p.bar_off = (int32_t)total;
@@ -232,7 +246,7 @@ static size_t layout_banded(BandedParams &p, int D, bool norm) {
   p.gamma_off = (int32_t)round_up(total, 16);
   total = p.gamma_off + (norm ? 4 * D * 4 : 0);
   p.items_off = (int32_t)round_up(total, 16);
-  const int G = kConsumers / (D / (16 / elem_bytes_of(p)));
+  const int G = kConsumers / (D / (2 * (16 / elem_bytes_of(p))));  // lanes per row: D / 2N
   total = p.items_off + (int64_t)((p.work_total + G - 1) / G) * kConsumers * 4;
   p.offs_off = (int32_t)round_up(total, 16);
   p.staged = p.batch <= kSmemSeqs;
@@ -240,41 +254,51 @@ static size_t layout_banded(BandedParams &p, int D, bool norm) {
   return (size_t)round_up(total, 128);
 }
 
-template <typename T, int D, bool NORM>
+template <typename T, int D, bool NORM, int CW, int LAG>
 static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStream_t st) {
   static ShapeCache cache;
-  auto kern = banded_store_kernel<T, D, NORM>;
-  const int occ = resident_ctas(kern, kPipeThreads, smem, cache);
+  auto kern = banded_store_kernel<T, D, NORM, CW, LAG>;
+  const int occ = resident_ctas(kern, pipe_threads<CW>(), smem, cache);
   if (occ <= 0) return ROPE_ERR_UNSUPPORTED;  // the stage ring does not fit
   const int64_t slots = (int64_t)sm_count() * occ;
   const int grid = (int)(slots < p.T ? slots : p.T);
-  kern<<<grid, kPipeThreads, smem, st>>>(p);
+  kern<<<grid, pipe_threads<CW>(), smem, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ROPE_OK : ROPE_ERR_CUDA;
 }
 
+template <typename T, int D, bool NORM>
+static rope_status_t launch_banded_s(const BandedShape &sh, const BandedParams &p, size_t smem,
+                                     cudaStream_t st) {
+  if (sh.cw == kLightShape.cw)
+    return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
+  return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag>(p, smem, st);
+}
+
 template <typename T, bool NORM>
-static rope_status_t launch_banded_d(int D, const BandedParams &p, size_t smem, cudaStream_t st) {
-  if (D == 64) return launch_banded_t<T, 64, NORM>(p, smem, st);
-  if (D == 128) return launch_banded_t<T, 128, NORM>(p, smem, st);
+static rope_status_t launch_banded_d(int D, const BandedShape &sh, const BandedParams &p,
+                                     size_t smem, cudaStream_t st) {
+  if (D == 64) return launch_banded_s<T, 64, NORM>(sh, p, smem, st);
+  if (D == 128) return launch_banded_s<T, 128, NORM>(sh, p, smem, st);
   if constexpr (sizeof(T) == 2)
-    if (D == 256) return launch_banded_t<T, 256, NORM>(p, smem, st);
+    if (D == 256) return launch_banded_s<T, 256, NORM>(sh, p, smem, st);
   return ROPE_ERR_UNSUPPORTED;
 }
 
 static rope_status_t launch_banded(int dtype, int D, bool norm, BandedParams &p,
                                    cudaStream_t st) {
   p.elem_bytes = elem_bytes(dtype);
-  const size_t smem = layout_banded(p, D, norm);
+  const BandedShape sh = pick_shape(p, norm);
+  const size_t smem = layout_banded(p, D, norm, sh);
   if (smem > 227 * 1024) return ROPE_ERR_UNSUPPORTED;
   if (dtype == ROPE_DTYPE_BF16)
-    return norm ? launch_banded_d<__nv_bfloat16, true>(D, p, smem, st)
-                : launch_banded_d<__nv_bfloat16, false>(D, p, smem, st);
+    return norm ? launch_banded_d<__nv_bfloat16, true>(D, sh, p, smem, st)
+                : launch_banded_d<__nv_bfloat16, false>(D, sh, p, smem, st);
   if (dtype == ROPE_DTYPE_F16)
-    return norm ? launch_banded_d<__half, true>(D, p, smem, st)
-                : launch_banded_d<__half, false>(D, p, smem, st);
+    return norm ? launch_banded_d<__half, true>(D, sh, p, smem, st)
+                : launch_banded_d<__half, false>(D, sh, p, smem, st);
   if (dtype == ROPE_DTYPE_F32)
-    return norm ? launch_banded_d<float, true>(D, p, smem, st)
-                : launch_banded_d<float, false>(D, p, smem, st);
+    return norm ? launch_banded_d<float, true>(D, sh, p, smem, st)
+                : launch_banded_d<float, false>(D, sh, p, smem, st);
   return ROPE_ERR_UNSUPPORTED;
 }
 
@@ -300,7 +324,10 @@ static rope_status_t launch_bshd_d(int D, const BshdParams &p, cudaStream_t st) 
   return ROPE_ERR_UNSUPPORTED;
 }
 
+constexpr int kRaddRing = 96 << 10;  // shared memory of a radd CTA's stage ring
+
 static size_t layout_radd(RaddParams &p, int D, int eb) {
+  const int kStageTarget = kRaddRing;
   p.stage_bytes = (int32_t)round_up(4LL * p.n_kv * D * eb, 128);
   int S = (int)(kStageTarget / p.stage_bytes);
   S = S < 2 ? 2 : (S > kMaxStages ? kMaxStages : S);
