@@ -6,9 +6,11 @@
 One step = one rope_split_store_paged_ragged call (RoPE of Q and K, split, paged K/V store)
 over the Llama-3-8B-shaped ragged prefill batch: 32 Q / 8 KV heads, head_dim 128, 8
 sequences with seeded lengths U[256, 2048], page_size 128, half-split RoPE, bf16.  Inputs are
-resident in HBM; a 256 MiB memset flushes L2 before every step, outside the timed events.
-`value` = tokens processed by all ranks / the max over ranks of the summed per-step device
-time (CUDA events on the launching stream).  Under torchrun every rank runs its own replica
+resident in HBM and larger than L2: the steps rotate over three separate copies of the
+workload (about 0.8 GB), launched back to back, so no step finds its inputs in L2 and every
+step pays for writing back the dirty lines its predecessor left.  `value` = tokens
+processed by all ranks / the max over ranks of the summed per-step device time (CUDA events
+on the launching stream).  Under torchrun every rank runs its own replica
 of the workload (its own seeded batch: weak scaling, no collective on the data path).
 
 Also printed (same JSON line): `e2e` (the same step through the Python binding with the
@@ -36,7 +38,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused RoPE+KV-store tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "tokens/s"
-FLUSH_BYTES = 256 << 20
+FLUSH_BYTES = 256 << 20   # L2 flush for the decode case's cold-cache figure
+REPLICAS = 3               # rotating copies of a workload: inputs larger than L2
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/rope_store.cu", "rope_paged_kv_b200/csrc/banded.cuh",
                   "rope_paged_kv_b200/csrc/common.cuh", "rope_paged_kv_b200/csrc/pipeline.cuh",
@@ -205,7 +208,14 @@ class Case:
     result copied back."""
 
 
-def make_case(name, seed, dev):
+def make_workload(name, seed):
+    import workloads as W
+    return {"llama3_8b_prefill": W.llama3_8b_prefill, "per_head_norm": W.per_head_norm,
+            "dual_band_minimax": W.dual_band_minimax, "radd_minimax": W.radd_minimax,
+            "decode_bshd": W.decode_bshd}[name](seed)
+
+
+def make_case(name, seed, dev, w=None):
     import ctypes
 
     import torch
@@ -241,7 +251,7 @@ def make_case(name, seed, dev):
         return t.contiguous().pin_memory()
 
     if name in ("llama3_8b_prefill", "per_head_norm"):
-        w = W.llama3_8b_prefill(seed) if name == "llama3_8b_prefill" else W.per_head_norm(seed)
+        w = w or make_workload(name, seed)
         kv = w.cache
         storage = d(kv.storage)
         cache = paged(kv, storage)
@@ -286,7 +296,7 @@ def make_case(name, seed, dev):
                     "rmsnorm": w.q_gamma is not None}
         c.workload = w
     elif name == "dual_band_minimax":
-        w = W.dual_band_minimax(seed)
+        w = w or make_workload(name, seed)
         inp, offs = d(w.input), d(w.offsets)
         ms, ist = d(w.main_cache.storage), d(w.index_cache.storage)
         g = [d(x) for x in w.gammas]
@@ -323,7 +333,7 @@ def make_case(name, seed, dev):
                     "batch": len(w.lengths)}
         c.workload = w
     elif name == "radd_minimax":
-        w = W.radd_minimax(seed)
+        w = w or make_workload(name, seed)
         st_, a, offs = d(w.cache.storage), d(w.a), d(w.offsets)
         cache = paged(w.cache, st_)
         c_kv = cache.c()
@@ -346,7 +356,7 @@ def make_case(name, seed, dev):
                     "page_size": w.cache.page_size, "batch": len(w.lengths)}
         c.workload = w
     elif name == "decode_bshd":
-        w = W.decode_bshd(seed)
+        w = w or make_workload(name, seed)
         kv = w.cache
         st_, out = d(kv.storage), d(w.output)
         cc = rs.ContCache(st_, None, d(kv.lookup_table), d(kv.cache_lengths), kv.n_kv_heads,
@@ -388,17 +398,32 @@ def make_case(name, seed, dev):
     return c
 
 
-def time_steps(torch, step, flush, k, stream):
-    """Device time (ms) of k calls of step(), each after an L2 flush outside its events."""
+def time_steps(torch, steps, k, stream, flush=None):
+    """Device time (ms) of k calls, step i calling steps[i % len(steps)], launched back to
+    back (each between its own pair of events); with `flush`, an L2 flush precedes every
+    call outside its events."""
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(k)]
     for i in range(k):
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         ev[i][0].record(stream)
-        step()
+        steps[i % len(steps)]()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     return sum(a.elapsed_time(b) for a, b in ev)
+
+
+def combine_ranks(torch, dist, tokens, dev_ms, e2e_ms, device):
+    """Whole-job figures: tokens summed over ranks, device times maxed over ranks (dist is
+    None for a single process)."""
+    tok = torch.tensor([float(tokens)], device=device, dtype=torch.float64)
+    times = torch.tensor([float(dev_ms), float(e2e_ms)], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(tok, op=dist.ReduceOp.SUM)
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    t = times.tolist()
+    return float(tok.item()), float(t[0]), float(t[1])
 
 
 def run_ours(args):
@@ -418,27 +443,28 @@ def run_ours(args):
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    # this rank's replica: its own seeded batch
-    case = make_case(args.workload, 1000 * rank, dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    # this rank's replica: its own seeded batch, staged REPLICAS times
+    w = make_workload(args.workload, 1000 * rank)
+    cases = [make_case(args.workload, 1000 * rank, dev, w) for _ in range(REPLICAS)]
+    case = cases[0]
     stream = torch.cuda.current_stream()
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(local))
+    steps = [c.step for c in cases]
 
     W_ = max(3, args.warmup)
-    for _ in range(W_):
-        flush.zero_()
-        case.step()
+    for i in range(W_):
+        steps[i % REPLICAS]()
     torch.cuda.synchronize()
     if args.workload != "radd_minimax":   # radd accumulates: its data stays valid anyway
-        assert int(case.err.item()) == 0, "device error bits set on the benchmark workload"
+        assert all(int(c.err.item()) == 0 for c in cases), "device error bits set"
 
     K = args.steps
     barrier()
     torch.cuda.synchronize()
     t0 = time.time()
-    dev_ms = time_steps(torch, case.step, flush, K, stream)
+    dev_ms = time_steps(torch, steps, K, stream)
     t1 = time.time()
     barrier()
 
@@ -447,22 +473,19 @@ def run_ours(args):
         case.e2e_step()
     barrier()
     torch.cuda.synchronize()
-    e2e_ms = time_steps(torch, case.e2e_step, flush, K_e2e, stream)
+    e2e_ms = time_steps(torch, [case.e2e_step], K_e2e, stream)
     barrier()
     sampler.stop()
+    del cases[1:]
+    torch.cuda.empty_cache()
 
-    tokens = torch.tensor([float(case.tokens)], device=dev, dtype=torch.float64)
-    times = torch.tensor([dev_ms, e2e_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(tokens, op=dist.ReduceOp.SUM)
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    tok_all = float(tokens.item())
-    dev_ms_max, e2e_ms_max = (float(x) for x in times.tolist())
+    tok_all, dev_ms_max, e2e_ms_max = combine_ranks(torch, dist if world > 1 else None,
+                                                    case.tokens, dev_ms, e2e_ms, dev)
 
     peak, peak_src = measured_peak()
     extras, cpu = {}, None
     if rank == 0 and world == 1 and not args.no_extras:
-        extras = run_entry_points(torch, dev, flush, stream, args.workload, peak)
+        extras = run_entry_points(torch, dev, stream, args.workload, peak)
         extras[args.workload] = summarize(case, dev_ms / K / 1e3, peak)
         cpu = cpu_baseline(args.workload)
     if world > 1:
@@ -480,8 +503,8 @@ def run_ours(args):
         "data": "synthetic (seeded, shapes of the named workload)",
         "config": dict({"workload": case.workload.name, "entry_point": case.entry_point,
                         "tokens_per_rank": case.tokens, "cache_dtype": "bf16",
-                        "l2": "flushed before every step (256 MiB memset outside the timed "
-                              "events)",
+                        "l2": f"inputs larger than L2: {REPLICAS} rotating copies of the "
+                              f"workload, launched back to back",
                         "parallelism": f"replicas x{world} (each rank its own batch, "
                                        f"no collective)"}, **case.config),
         "gpu_launches": K,
@@ -519,29 +542,27 @@ def summarize(case, sec, peak):
             "frac_of_measured_hbm": round(gbs / peak, 3)}
 
 
-def run_entry_points(torch, dev, flush, stream, headline, peak, reps=20):
+def run_entry_points(torch, dev, stream, headline, peak, reps=30):
     """Every other named workload, timed the same way (N=1 only; reported beside the
     headline, not instead of it)."""
     out = {}
     for name in WORKLOADS:
         if name == headline:
             continue
-        case = make_case(name, 0, dev)
-        for _ in range(3):
-            flush.zero_()
-            case.step()
-        sec = time_steps(torch, case.step, flush, reps, stream) / reps / 1e3
-        out[name] = summarize(case, sec, peak)
+        w = make_workload(name, 0)
+        cases = [make_case(name, 0, dev, w) for _ in range(REPLICAS)]
+        steps = [c.step for c in cases]
+        for i in range(3):
+            steps[i % REPLICAS]()
+        sec = time_steps(torch, steps, reps, stream) / reps / 1e3
+        out[name] = summarize(cases[0], sec, peak)
         if name == "decode_bshd":
-            # back-to-back launches without the flush (the decode step's L2-warm case)
-            a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            for _ in range(50):
-                case.step()
-            b0.record(stream)
-            torch.cuda.synchronize()
-            out[name]["us_per_launch_back_to_back_l2_warm"] = round(a0.elapsed_time(b0) / 50 * 1e3, 2)
-        del case
+            # the decode batch is L2-sized: also the cold figure, L2 flushed before each call
+            flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+            cold = time_steps(torch, steps, reps, stream, flush) / reps / 1e3
+            out[name]["us_per_launch_l2_flushed"] = round(cold * 1e6, 2)
+            del flush
+        del cases, steps
         torch.cuda.empty_cache()
     return out
 

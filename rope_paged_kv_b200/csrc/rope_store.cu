@@ -25,7 +25,13 @@ constexpr int kMaxStages = 8;
 struct BandedShape {
   int cw, lag, ring_kb;
 };
-constexpr BandedShape kLightShape = {4, 2, 64};  // <= 64 head rows of Q+K per token, no norm
+#ifndef ROPE_LIGHT_CW
+#define ROPE_LIGHT_CW 4
+#define ROPE_LIGHT_LAG 2
+#define ROPE_LIGHT_RING 64
+#endif
+// <= 64 Q+K head rows a token, no norm
+constexpr BandedShape kLightShape = {ROPE_LIGHT_CW, ROPE_LIGHT_LAG, ROPE_LIGHT_RING};
 constexpr BandedShape kHeavyShape = {8, 0, 96};  // RMSNorm or many heads
 
 static BandedShape pick_shape(const BandedParams &p, bool norm) {

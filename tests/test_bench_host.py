@@ -1,0 +1,69 @@
+"""Host-side logic of bench.py that needs no GPU: the multi-rank reduction (two gloo ranks on
+the CPU) and the reference arm (the CPU oracle) with its JSON line."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # each rank: its own token count and device times
+        out = bench.combine_ranks(torch, dist, tokens=100 + rank, dev_ms=2.0 + rank,
+                                  e2e_ms=10.0 - rank, device=torch.device("cpu"))
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_combine_ranks_sums_tokens_and_takes_max_time_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(2):
+        assert results[r] == (201.0, 3.0, 10.0)
+
+
+def test_combine_ranks_single_process():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.combine_ranks(torch, None, 7, 1.5, 2.5, torch.device("cpu")) == (7.0, 1.5, 2.5)
+
+
+def test_reference_arm_prints_one_json_line():
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                       timeout=600, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["unit"] == "tokens/s" and j["value"] > 0
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
+    assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["higher_is_better"] is True
+    assert j["steps"] == 2 and j["warmup"] >= 3
