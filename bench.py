@@ -57,6 +57,13 @@ def parse_args():
                     help="the named workload timed as the main line (default: the headline)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other entry points and the CPU baseline")
+    ap.add_argument("--overlap", type=int, choices=[0, 1, 2], default=2,
+                    help="launch overlap of consecutive calls: 0 off, 1 programmatic "
+                         "dependent launch, 2 the same with descriptor arrays read early "
+                         "(valid here: no kernel writes them)")
+    ap.add_argument("--schedule", choices=["claimed", "static"], default="claimed",
+                    help="token schedule of the staged kernels: claimed tail (a scheduling "
+                         "workspace) or static")
     return ap.parse_args()
 
 
@@ -215,7 +222,7 @@ def make_workload(name, seed):
             "decode_bshd": W.decode_bshd}[name](seed)
 
 
-def make_case(name, seed, dev, w=None):
+def make_case(name, seed, dev, w=None, sched=True):
     import ctypes
 
     import torch
@@ -238,6 +245,9 @@ def make_case(name, seed, dev, w=None):
     c = Case()
     c.name, c.entry_point = name, WORKLOADS[name]
     c.err = torch.zeros(1, dtype=torch.int32, device=dev)
+    # scheduling workspace of the staged entry points (None: the static token schedule)
+    c.sched = rs.sched_workspace(dev) if sched else None
+    sched_ptr = None if c.sched is None else c.sched.data_ptr()
     keep = []
 
     def bind(fn, args, where):
@@ -262,31 +272,33 @@ def make_case(name, seed, dev, w=None):
         if w.q_gamma is None:
             args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
                     offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), w.layer_idx,
-                    q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(), stream.cuda_stream)
+                    q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(), sched_ptr,
+                    stream.cuda_stream)
             c.step = bind(lib.rope_split_store_paged_ragged, args, c.entry_point)
 
             def call():
                 rs.rope_split_store_paged_ragged(qkv, w.n_q_heads, offs, fr, cache, w.layer_idx,
-                                                 q_out, c.err)
+                                                 q_out, c.err, sched=c.sched)
         else:
             qg, kg = d(w.q_gamma), d(w.k_gamma)
             args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
                     offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), qg.data_ptr(),
                     kg.data_ptr(), ctypes.c_float(w.epsilon), ctypes.c_float(w.weight_offset), 1,
                     w.layer_idx, q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(),
-                    stream.cuda_stream)
+                    sched_ptr, stream.cuda_stream)
             c.step = bind(lib.fused_qk_rmsnorm_rope_paged, args, c.entry_point)
 
             def call():
                 rs.fused_qk_rmsnorm_rope_paged(qkv, w.n_q_heads, offs, fr, cache, qg, kg,
                                                w.epsilon, w.weight_offset, w.layer_idx, q_out,
-                                               True, c.err)
+                                               True, c.err, sched=c.sched)
         c.tokens = w.total_tokens
         c.alg_bytes = bytes_ragged(w)
         c.e2e_in = [(pinned(w.qkv), qkv), (pinned(w.offsets), offs),
                     (pinned(kv.cache_lengths), cache.cache_lengths),
                     (pinned(kv.page_table), cache.page_table)]
         c.e2e_out = [(q_out, torch.empty(q_out.shape, dtype=q_out.dtype).pin_memory())]
+        c.outputs = [q_out, storage]
         c.call = call
         c.config = {"n_q_heads": w.n_q_heads, "n_kv_heads": kv.n_kv_heads,
                     "head_dim": kv.head_dim, "page_size": kv.page_size,
@@ -310,12 +322,13 @@ def make_case(name, seed, dev, w=None):
         keep += [mb, ib, c_f]
         args = (ctypes.byref(mb), ctypes.byref(ib), offs.data_ptr(), offs.shape[0] - 1,
                 w.total_tokens, ctypes.byref(c_f), ctypes.c_float(w.weight_offset), 1,
-                w.layer_idx, c.err.data_ptr(), stream.cuda_stream)
+                w.layer_idx, c.err.data_ptr(), sched_ptr, stream.cuda_stream)
         c.step = bind(lib.fused_dual_qk_rmsnorm_rope_paged, args, c.entry_point)
 
         def call():
             rs.fused_dual_qk_rmsnorm_rope_paged(main, index, offs, w.total_tokens, fr,
-                                                w.weight_offset, w.layer_idx, True, c.err)
+                                                w.weight_offset, w.layer_idx, True, c.err,
+                                                sched=c.sched)
         c.call = call
         c.tokens = w.total_tokens
         c.alg_bytes = bytes_dual(w)
@@ -324,6 +337,7 @@ def make_case(name, seed, dev, w=None):
                     (pinned(w.main_cache.page_table), main.cache.page_table),
                     (pinned(w.index_cache.cache_lengths), index.cache.cache_lengths),
                     (pinned(w.index_cache.page_table), index.cache.page_table)]
+        c.outputs = [qm, qi, ms, ist]
         c.e2e_out = [(qm, torch.empty(qm.shape, dtype=qm.dtype).pin_memory()),
                      (qi, torch.empty(qi.shape, dtype=qi.dtype).pin_memory())]
         c.config = {"main_heads": [w.main_q_heads, w.main_cache.n_kv_heads],
@@ -339,12 +353,13 @@ def make_case(name, seed, dev, w=None):
         c_kv = cache.c()
         keep.append(c_kv)
         args = (a.data_ptr(), a.stride(0), a.shape[0], ctypes.byref(c_kv), offs.data_ptr(),
-                offs.shape[0] - 1, w.batch_offset, w.layer_idx, c.err.data_ptr(),
+                offs.shape[0] - 1, w.batch_offset, w.layer_idx, c.err.data_ptr(), sched_ptr,
                 stream.cuda_stream)
         c.step = bind(lib.kv_cache_radd, args, c.entry_point)
 
         def call():
-            rs.kv_cache_radd(a, cache, offs, w.batch_offset, w.layer_idx, c.err)
+            rs.kv_cache_radd(a, cache, offs, w.batch_offset, w.layer_idx, c.err,
+                             sched=c.sched)
         c.call = call
         c.tokens = w.a.shape[0]
         c.alg_bytes = bytes_radd(w)
@@ -352,6 +367,7 @@ def make_case(name, seed, dev, w=None):
                     (pinned(w.cache.cache_lengths), cache.cache_lengths),
                     (pinned(w.cache.page_table), cache.page_table)]
         c.e2e_out = [(c.err, torch.empty(1, dtype=torch.int32).pin_memory())]
+        c.outputs = [st_]
         c.config = {"n_kv_heads": w.cache.n_kv_heads, "head_dim": w.cache.head_dim,
                     "page_size": w.cache.page_size, "batch": len(w.lengths)}
         c.workload = w
@@ -398,10 +414,19 @@ def make_case(name, seed, dev, w=None):
     return c
 
 
-def time_steps(torch, steps, k, stream, flush=None):
+def time_steps(torch, steps, k, stream, flush=None, per_launch=False):
     """Device time (ms) of k calls, step i calling steps[i % len(steps)], launched back to
-    back (each between its own pair of events); with `flush`, an L2 flush precedes every
-    call outside its events."""
+    back between one pair of events on `stream`.  per_launch: each call between its own
+    pair of events instead (an isolated launch: nothing overlaps it), the sum returned; with
+    `flush`, an L2 flush precedes every call outside its events."""
+    if not per_launch:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(k):
+            steps[i % len(steps)]()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(k)]
     for i in range(k):
@@ -443,9 +468,13 @@ def run_ours(args):
         if world > 1:
             dist.barrier(device_ids=[local])
 
+    import rope_paged_kv_b200 as rs
+    rs.set_launch_overlap(args.overlap)
+    use_sched = args.schedule == "claimed"
     # this rank's replica: its own seeded batch, staged REPLICAS times
     w = make_workload(args.workload, 1000 * rank)
-    cases = [make_case(args.workload, 1000 * rank, dev, w) for _ in range(REPLICAS)]
+    cases = [make_case(args.workload, 1000 * rank, dev, w, use_sched)
+             for _ in range(REPLICAS)]
     case = cases[0]
     stream = torch.cuda.current_stream()
     props = torch.cuda.get_device_properties(dev)
@@ -459,6 +488,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     if args.workload != "radd_minimax":   # radd accumulates: its data stays valid anyway
         assert all(int(c.err.item()) == 0 for c in cases), "device error bits set"
+    assert all(c.sched is None or not c.sched.any().item() for c in cases), \
+        "a scheduling workspace was not returned to zero"
 
     K = args.steps
     barrier()
@@ -483,9 +514,10 @@ def run_ours(args):
                                                     case.tokens, dev_ms, e2e_ms, dev)
 
     peak, peak_src = measured_peak()
-    extras, cpu = {}, None
+    extras, cpu, modes = {}, None, None
     if rank == 0 and world == 1 and not args.no_extras:
-        extras = run_entry_points(torch, dev, stream, args.workload, peak)
+        modes = launch_modes(torch, dev, stream, args, w, peak)
+        extras = run_entry_points(torch, dev, stream, args.workload, peak, use_sched)
         extras[args.workload] = summarize(case, dev_ms / K / 1e3, peak)
         cpu = cpu_baseline(args.workload)
     if world > 1:
@@ -505,6 +537,9 @@ def run_ours(args):
                         "tokens_per_rank": case.tokens, "cache_dtype": "bf16",
                         "l2": f"inputs larger than L2: {REPLICAS} rotating copies of the "
                               f"workload, launched back to back",
+                        "overlap": OVERLAP_NAMES[args.overlap],
+                        "schedule": "claimed tail (scheduling workspace)" if use_sched
+                                    else "static",
                         "parallelism": f"replicas x{world} (each rank its own batch, "
                                        f"no collective)"}, **case.config),
         "gpu_launches": K,
@@ -522,6 +557,8 @@ def run_ours(args):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if modes:
+        line["launch_modes"] = modes
     if extras:
         line["entry_points"] = extras
     print(json.dumps(line), flush=True)
@@ -542,7 +579,35 @@ def summarize(case, sec, peak):
             "frac_of_measured_hbm": round(gbs / peak, 3)}
 
 
-def run_entry_points(torch, dev, stream, headline, peak, reps=30):
+OVERLAP_NAMES = {0: "off", 1: "pdl", 2: "pdl_early_metadata"}
+
+
+def launch_modes(torch, dev, stream, args, w, peak, reps=300):
+    """The headline workload under every launch-overlap mode and both token schedules
+    (reported beside the headline): us per launch back to back, plus one isolated launch
+    (its own events, no overlap)."""
+    import rope_paged_kv_b200 as rs
+    out = {}
+    for use_sched in (True, False):
+        cases = [make_case(args.workload, 0, dev, w, use_sched) for _ in range(REPLICAS)]
+        steps = [c.step for c in cases]
+        tag = "claimed" if use_sched else "static"
+        for mode in (0, 1, 2):
+            rs.set_launch_overlap(mode)
+            for i in range(6):
+                steps[i % REPLICAS]()
+            sec = time_steps(torch, steps, reps, stream) / reps / 1e3
+            out[f"{tag}/{OVERLAP_NAMES[mode]}"] = summarize(cases[0], sec, peak)["us_per_launch"]
+        rs.set_launch_overlap(0)
+        sec = time_steps(torch, steps, reps, stream, per_launch=True) / reps / 1e3
+        out[f"{tag}/isolated_launch"] = round(sec * 1e6, 2)
+        del cases, steps
+        torch.cuda.empty_cache()
+    rs.set_launch_overlap(args.overlap)
+    return {"unit": "us per launch", "workload": w.name, **out}
+
+
+def run_entry_points(torch, dev, stream, headline, peak, use_sched, reps=30):
     """Every other named workload, timed the same way (N=1 only; reported beside the
     headline, not instead of it)."""
     out = {}
@@ -550,16 +615,17 @@ def run_entry_points(torch, dev, stream, headline, peak, reps=30):
         if name == headline:
             continue
         w = make_workload(name, 0)
-        cases = [make_case(name, 0, dev, w) for _ in range(REPLICAS)]
+        cases = [make_case(name, 0, dev, w, use_sched) for _ in range(REPLICAS)]
         steps = [c.step for c in cases]
         for i in range(3):
             steps[i % REPLICAS]()
         sec = time_steps(torch, steps, reps, stream) / reps / 1e3
         out[name] = summarize(cases[0], sec, peak)
         if name == "decode_bshd":
-            # the decode batch is L2-sized: also the cold figure, L2 flushed before each call
+            # the decode batch is L2-sized: also the cold figure, an isolated launch with L2
+            # flushed before each call
             flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-            cold = time_steps(torch, steps, reps, stream, flush) / reps / 1e3
+            cold = time_steps(torch, steps, reps, stream, flush, per_launch=True) / reps / 1e3
             out[name]["us_per_launch_l2_flushed"] = round(cold * 1e6, 2)
             del flush
         del cases, steps

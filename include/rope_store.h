@@ -34,6 +34,24 @@
  *           input_row_offsets is not a partition of [0, total_tokens) (first entry 0,
  *           non-decreasing, last entry total_tokens) the whole call writes nothing.  The
  *           kernels never trap and never wait on other blocks.
+ * Schedule. The calls that stage token rows (the three paged stores and kv_cache_radd)
+ *           take `sched`: NULL, or ROPE_SCHED_WORDS uint32 words of device memory (the
+ *           scheduling workspace).  With NULL every CTA processes a fixed strided share of
+ *           the tokens.  With a workspace each CTA takes most of its share that way and
+ *           then claims the remaining tokens in small chunks from a counter in the
+ *           workspace, so that CTAs which get more memory bandwidth take more of the tail;
+ *           the results are the same either way.  The words must be zero before the first
+ *           call that uses them (e.g. cudaMemsetAsync once after allocating); every call
+ *           leaves them zero when it completes.  Calls that can run at the same time (on
+ *           different streams) need separate workspaces; calls in one stream may share one.
+ * Overlap.  By default (ROPE_OVERLAP_PDL) every kernel is launched as a programmatic
+ *           dependent of the previous kernel in its stream: its CTAs may start while that
+ *           kernel finishes, and wait for it to complete before they touch global memory.
+ *           ROPE_OVERLAP_PDL_EARLY_METADATA additionally reads the descriptor arrays
+ *           (input_row_offsets, cache_lengths, page tables, lookup tables, valid_lengths,
+ *           gammas) before that wait: only valid when no kernel still running ahead in the
+ *           stream writes them (e.g. they were uploaded before the layer's kernels were
+ *           queued).  ROPE_OVERLAP_OFF launches plainly.  See rope_set_launch_overlap.
  */
 #ifndef ROPE_STORE_H
 #define ROPE_STORE_H
@@ -63,6 +81,15 @@ typedef enum { ROPE_DTYPE_BF16 = 0, ROPE_DTYPE_F16 = 1, ROPE_DTYPE_F32 = 2 } rop
 #define ROPE_DEVERR_PAGE_ID 0x8u     /* page-table entry >= num_pages */
 #define ROPE_DEVERR_BATCH 0x10u      /* sequence (+ batch_offset) >= n_seqs, or slot >= num_slots */
 #define ROPE_DEVERR_TIMEOUT 0x20u    /* an internal pipeline wait gave up (the call is incomplete) */
+
+/* uint32 words of a scheduling workspace (see Schedule above) */
+#define ROPE_SCHED_WORDS 2
+
+typedef enum {
+  ROPE_OVERLAP_OFF = 0,               /* plain launches */
+  ROPE_OVERLAP_PDL = 1,               /* programmatic dependent launch (the default) */
+  ROPE_OVERLAP_PDL_EARLY_METADATA = 2 /* as PDL, descriptor arrays read before the wait */
+} rope_overlap_t;
 
 /* freqs_cis [max_seq_len, rope_dim], row-major, contiguous.  Row p holds rope_dim/2
  * pairs (cos, sin): column 2i is cos and 2i+1 is sin of pair i's angle at position p (the
@@ -167,7 +194,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
                                             const rope_freqs_t *freqs,
                                             const rope_paged_cache_t *kv, uint32_t layer_idx,
                                             void *q_out, int64_t q_out_row_stride,
-                                            uint32_t *err_word, rope_stream_t stream);
+                                            uint32_t *err_word, uint32_t *sched,
+                                            rope_stream_t stream);
 
 /* fused_qk_rmsnorm_rope_paged -- the single-band per-head RMSNorm + RoPE + paged store that
  * the fused_dual_qk_rms_norm_rope_ragged_paged page fuses twice (its first paragraph).
@@ -186,7 +214,7 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
                                           float weight_offset, int32_t multiply_before_cast,
                                           uint32_t layer_idx, void *q_out,
                                           int64_t q_out_row_stride, uint32_t *err_word,
-                                          rope_stream_t stream);
+                                          uint32_t *sched, rope_stream_t stream);
 
 /* fused_dual_qk_rmsnorm_rope_paged -- fused_dual_qk_rms_norm_rope_ragged_paged page
  * (signature and both paragraphs): the main band and the index band in ONE launch.  Both
@@ -203,7 +231,8 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
                                                int32_t batch, int32_t total_tokens,
                                                const rope_freqs_t *freqs, float weight_offset,
                                                int32_t multiply_before_cast, uint32_t layer_idx,
-                                               uint32_t *err_word, rope_stream_t stream);
+                                               uint32_t *err_word, uint32_t *sched,
+                                               rope_stream_t stream);
 
 /* qk_rope_bshd_continuous -- generic_fused_qk_rope_bshd_continuous_batch page (signature,
  * description, Args).  q_proj and output: [batch, seq_len, n_q_heads, head_dim],
@@ -229,10 +258,16 @@ rope_status_t qk_rope_bshd_continuous(const void *q_proj, int32_t batch, int32_t
 rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_tokens,
                             const rope_paged_cache_t *kv, const uint32_t *input_row_offsets,
                             int32_t batch, uint32_t batch_offset, uint32_t layer_idx,
-                            uint32_t *err_word, rope_stream_t stream);
+                            uint32_t *err_word, uint32_t *sched, rope_stream_t stream);
 
 /* A static, human-readable name of a status code. */
 const char *rope_status_string(rope_status_t status);
+
+/* Launch-overlap mode (rope_overlap_t) of every launch that follows, process-wide; not a
+ * kernel of the method but a launch option (Overlap above).  Returns ROPE_ERR_INVALID_ARG
+ * for an unknown mode, leaving the mode as it was. */
+rope_status_t rope_set_launch_overlap(int32_t mode);
+int32_t rope_get_launch_overlap(void);
 
 #ifdef __cplusplus
 }

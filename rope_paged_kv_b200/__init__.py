@@ -18,6 +18,14 @@ PagedCache(k, v, page_table, cache_lengths, n_kv_heads, head_dim, page_size, num
 ContCache(k, v, lookup_table, cache_lengths, n_kv_heads, head_dim, num_slots, num_layers,
           max_seq_len, slot_stride, layer_stride, pos_stride, head_stride)
 NormBand(input, q_col, k_col, v_col, n_q_heads, cache, q_gamma, k_gamma, epsilon, q_out)
+
+Scheduling workspace and launch overlap
+---------------------------------------
+The staged entry points take ``sched``: None (a static token schedule) or a device tensor of
+at least SCHED_WORDS int32 words that is zero before its first use (``sched_workspace()``);
+every call leaves it zero.  Concurrent calls on different streams need separate
+workspaces.  ``set_launch_overlap(mode)`` picks how launches overlap the previous kernel of
+the stream (OVERLAP_OFF, OVERLAP_PDL = default, OVERLAP_PDL_EARLY_METADATA).
 """
 from __future__ import annotations
 
@@ -36,6 +44,8 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "rope_store.h")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA = 0, 1, 2, 3
 DEVERR_ROW_OFFSETS, DEVERR_POSITION, DEVERR_PAGE_INDEX = 0x1, 0x2, 0x4
 DEVERR_PAGE_ID, DEVERR_BATCH, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
+SCHED_WORDS = 2
+OVERLAP_OFF, OVERLAP_PDL, OVERLAP_PDL_EARLY_METADATA = 0, 1, 2
 
 _DTYPE_CODE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 
@@ -79,18 +89,24 @@ class c_norm_band(ctypes.Structure):
 
 _P = ctypes.POINTER
 _lib.rope_split_store_paged_ragged.argtypes = [
-    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp, _vp]
+    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp,
+    _vp, _vp]
 _lib.fused_qk_rmsnorm_rope_paged.argtypes = [
     _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _vp, _vp, _f32, _f32,
-    _i32, _u32, _vp, _i64, _vp, _vp]
+    _i32, _u32, _vp, _i64, _vp, _vp, _vp]
 _lib.fused_dual_qk_rmsnorm_rope_paged.argtypes = [
-    _P(c_norm_band), _P(c_norm_band), _vp, _i32, _i32, _P(c_freqs), _f32, _i32, _u32, _vp, _vp]
+    _P(c_norm_band), _P(c_norm_band), _vp, _i32, _i32, _P(c_freqs), _f32, _i32, _u32, _vp,
+    _vp, _vp]
 _lib.qk_rope_bshd_continuous.argtypes = [
     _vp, _i32, _i32, _i32, _i32, _P(c_cont_cache), _P(c_freqs), _u32, _vp, _vp, _vp, _vp]
 _lib.kv_cache_radd.argtypes = [
-    _vp, _i64, _i32, _P(c_paged_cache), _vp, _i32, _u32, _u32, _vp, _vp]
+    _vp, _i64, _i32, _P(c_paged_cache), _vp, _i32, _u32, _u32, _vp, _vp, _vp]
+_lib.rope_set_launch_overlap.argtypes = [_i32]
+_lib.rope_get_launch_overlap.argtypes = []
+_lib.rope_get_launch_overlap.restype = _i32
 for _f in ("rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
-           "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd"):
+           "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd",
+           "rope_set_launch_overlap"):
     getattr(_lib, _f).restype = ctypes.c_int
 _lib.rope_status_string.argtypes = [ctypes.c_int]
 _lib.rope_status_string.restype = ctypes.c_char_p
@@ -100,7 +116,8 @@ def header_functions() -> list:
     """Names of the functions include/rope_store.h declares."""
     with open(HEADER_PATH) as f:
         text = f.read()
-    return re.findall(r"^(?:rope_status_t|const char \*)\s*\n?\s*\**(\w+)\(", text, re.M)
+    return re.findall(r"^(?:rope_status_t|int32_t|const char \*)\s*\n?\s*\**(\w+)\(", text,
+                      re.M)
 
 
 class RopeError(RuntimeError):
@@ -123,6 +140,30 @@ def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _sched(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if (t.dtype not in (torch.int32, torch.uint32) or not t.is_contiguous()
+            or t.numel() < SCHED_WORDS or not t.is_cuda):
+        raise ValueError(f"sched must be a contiguous CUDA int32 tensor of >= {SCHED_WORDS} words")
+    return t.data_ptr()
+
+
+def sched_workspace(device=None) -> torch.Tensor:
+    """A zeroed scheduling workspace for the staged entry points."""
+    return torch.zeros(SCHED_WORDS, dtype=torch.int32,
+                       device=device if device is not None else torch.cuda.current_device())
+
+
+def set_launch_overlap(mode: int) -> None:
+    """How launches overlap the previous kernel of their stream (process-wide)."""
+    _check(_lib.rope_set_launch_overlap(int(mode)), "rope_set_launch_overlap")
+
+
+def get_launch_overlap() -> int:
+    return int(_lib.rope_get_launch_overlap())
 
 
 def _row_stride(t: torch.Tensor) -> int:
@@ -229,40 +270,41 @@ class NormBand:
 
 def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
                                   kv: PagedCache, layer_idx, q_out, err_word=None,
-                                  stream=None) -> None:
+                                  stream=None, sched=None) -> None:
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.rope_split_store_paged_ragged(
         qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
-        _row_stride(q_out), _ptr(err_word), _stream(stream)), "rope_split_store_paged_ragged")
+        _row_stride(q_out), _ptr(err_word), _sched(sched), _stream(stream)),
+        "rope_split_store_paged_ragged")
 
 
 def fused_qk_rmsnorm_rope_paged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
                                 kv: PagedCache, q_gamma, k_gamma, epsilon, weight_offset,
                                 layer_idx, q_out, multiply_before_cast=True, err_word=None,
-                                stream=None) -> None:
+                                stream=None, sched=None) -> None:
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.fused_qk_rmsnorm_rope_paged(
         qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), q_gamma.data_ptr(),
         k_gamma.data_ptr(), epsilon, weight_offset, int(bool(multiply_before_cast)), layer_idx,
-        q_out.data_ptr(), _row_stride(q_out), _ptr(err_word), _stream(stream)),
+        q_out.data_ptr(), _row_stride(q_out), _ptr(err_word), _sched(sched), _stream(stream)),
         "fused_qk_rmsnorm_rope_paged")
 
 
 def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: NormBand,
                                      input_row_offsets, total_tokens, freqs: Freqs,
                                      weight_offset, layer_idx, multiply_before_cast=True,
-                                     err_word=None, stream=None) -> None:
+                                     err_word=None, stream=None, sched=None) -> None:
     offs = _idx(input_row_offsets)
     keep: list = []
     m, i, f = main_band.c(keep), index_band.c(keep), freqs.c()
     _check(_lib.fused_dual_qk_rmsnorm_rope_paged(
         ctypes.byref(m), ctypes.byref(i), offs.data_ptr(), offs.shape[0] - 1, total_tokens,
         ctypes.byref(f), weight_offset, int(bool(multiply_before_cast)), layer_idx,
-        _ptr(err_word), _stream(stream)), "fused_dual_qk_rmsnorm_rope_paged")
+        _ptr(err_word), _sched(sched), _stream(stream)), "fused_dual_qk_rmsnorm_rope_paged")
 
 
 def qk_rope_bshd_continuous(q_proj, kv: ContCache, freqs: Freqs, layer_idx, valid_lengths,
@@ -278,13 +320,13 @@ def qk_rope_bshd_continuous(q_proj, kv: ContCache, freqs: Freqs, layer_idx, vali
 
 
 def kv_cache_radd(a, kv: PagedCache, input_row_offsets, batch_offset, layer_idx,
-                  err_word=None, stream=None) -> None:
+                  err_word=None, stream=None, sched=None) -> None:
     offs = _idx(input_row_offsets)
     c = kv.c()
     _check(_lib.kv_cache_radd(
         a.data_ptr(), _row_stride(a), a.shape[0], ctypes.byref(c), offs.data_ptr(),
-        offs.shape[0] - 1, batch_offset, layer_idx, _ptr(err_word), _stream(stream)),
-        "kv_cache_radd")
+        offs.shape[0] - 1, batch_offset, layer_idx, _ptr(err_word), _sched(sched),
+        _stream(stream)), "kv_cache_radd")
 
 
 def raw_library() -> ctypes.CDLL:

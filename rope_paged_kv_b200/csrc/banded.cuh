@@ -4,11 +4,14 @@
 //
 // Persistent CTAs, one ring of S shared-memory stages each; a token's row lives in one
 // stage from load to store, and the bulk-copy (TMA) engine moves it both ways:
-//   warp 0, producer:  for 32 tokens at a time each lane resolves one token (sequence by
-//                      binary search over the staged input_row_offsets, position,
-//                      page-table translation); then, token by token, it waits for a free
-//                      stage, publishes the metadata and bulk-copies the token's Q | K | V
-//                      head blocks of every band plus each band's freqs_cis row into it;
+//   warp 0, producer:  for up to 32 tokens at a time each lane resolves one token
+//                      (sequence by binary search over the staged input_row_offsets,
+//                      position, page-table translation); then, token by token, it waits
+//                      for a free stage, publishes the metadata and bulk-copies the token's
+//                      Q | K | V head blocks of every band plus each band's freqs_cis row
+//                      into it.  Its tokens are a static strided share and, when the caller
+//                      gives a workspace, chunks claimed from a counter after that (see
+//                      static_tokens); a stop marker in the next stage ends the CTA;
 //   warps 2.., consumers: per token, the Q and K head rows are spread over lane groups of
 //                      L = head_dim / vector lanes; each lane normalises (shuffle reduction
 //                      over its group) and rotates its 16 bytes (a half-split partner's 16
@@ -53,6 +56,8 @@ struct BandDev {
 struct BandedParams {
   BandDev band[2];
   int32_t n_bands;
+  int32_t overlap;   // launch-overlap mode (kOverlap*)
+  uint32_t *sched;   // claim counter + finished CTAs, or nullptr for a static schedule
   int32_t work0, work_total;  // Q + K head rows of band 0, of both bands
   const uint32_t *offs;
   int32_t batch, T;
@@ -76,6 +81,8 @@ struct StageMeta {
   int64_t kv_base[2];
   int32_t pos[2];
   int32_t ok[2];
+  int32_t tok;   // the token held by the stage
+  int32_t stop;  // no token: the CTA's work is done
 };
 
 // This lane's (cos, sin) for a token from the staged freqs_cis row F (element type fdt).
@@ -220,6 +227,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) grid_dep_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < p.S; ++s) {
       mbar_init(&full[s], 1);
@@ -229,6 +237,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
     s_abort = 0;
     fence_mbar_init();
   }
+  if (p.overlap != kOverlapEarlyMeta) grid_dep_wait();
   const bool good = stage_offsets(p.offs, p.batch, p.T, p.staged, s_offs);
   if (p.staged)
     for (int i = tid; i < p.n_bands * p.batch; i += kPipeThreads) {
@@ -243,7 +252,11 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
       s_gamma[i] = static_cast<float>(g[d]) + p.weight_offset;
     }
   if (!__syncthreads_and(good)) {
-    if (tid == 0) raise(p.err, ROPE_DEVERR_ROW_OFFSETS);
+    grid_dep_wait();
+    if (tid == 0) {
+      raise(p.err, ROPE_DEVERR_ROW_OFFSETS);
+      if (p.sched != nullptr) sched_release(p.sched);
+    }
     return;
   }
   const uint32_t *offs = p.staged ? s_offs : p.offs;
@@ -252,35 +265,47 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer --
+    const bool dyn = p.sched != nullptr;
+    const int n_static = static_tokens(p.T, n_local, dyn);
+    const int dyn0 = n_static * (int)gridDim.x;  // first claimed token
     int issued = 0;
     bool aborted = false;
-    for (int c = 0; c < n_local && !aborted; c += 32) {
-      StageMeta m{};
-      const int i = c + lane;
-      if (i < n_local) {
-        const uint32_t tok = blockIdx.x + (uint32_t)i * gridDim.x;
-        const int b = find_seq(offs, p.batch, tok);
-        const uint32_t t = tok - offs[b];
-        uint32_t e_all = 0;
+    bool waited = p.overlap != kOverlapEarlyMeta;  // otherwise done at the top
+    // This lane's token (tok < 0: none) resolved into m; returns its error bits, raised by
+    // the caller once the predecessors are done (error words may be reset by one).
+    auto resolve = [&](int tok, StageMeta &m) -> uint32_t {
+      m = StageMeta{};
+      m.tok = tok;
+      if (tok < 0) return 0u;
+      const int b = find_seq(offs, p.batch, (uint32_t)tok);
+      const uint32_t t = (uint32_t)tok - offs[b];
+      uint32_t e_all = 0;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          if (k >= p.n_bands) break;
-          const BandDev &bd = k ? p.band[1] : p.band[0];
-          const uint32_t cl = p.staged ? s_cl[k * p.batch + b] : __ldg(bd.cache.cache_lengths + b);
-          const uint64_t pos = (uint64_t)cl + t;
-          int64_t base = 0;
-          const uint32_t e = pos >= p.rope.max_seq_len
-                                 ? ROPE_DEVERR_POSITION
-                                 : translate(bd.cache, p.layer, (uint64_t)b, pos, &base);
-          m.ok[k] = (e == 0);
-          m.kv_base[k] = base;
-          m.pos[k] = (int32_t)(e == 0 ? pos : 0);
-          e_all |= e;
-        }
-        raise(p.err, e_all);
+      for (int k = 0; k < 2; ++k) {
+        if (k >= p.n_bands) break;
+        const BandDev &bd = k ? p.band[1] : p.band[0];
+        const uint32_t cl = p.staged ? s_cl[k * p.batch + b] : __ldg(bd.cache.cache_lengths + b);
+        const uint64_t pos = (uint64_t)cl + t;
+        int64_t base = 0;
+        const uint32_t e = pos >= p.rope.max_seq_len
+                               ? ROPE_DEVERR_POSITION
+                               : translate(bd.cache, p.layer, (uint64_t)b, pos, &base);
+        m.ok[k] = (e == 0);
+        m.kv_base[k] = base;
+        m.pos[k] = (int32_t)(e == 0 ? pos : 0);
+        e_all |= e;
       }
-      const int cnt = min(32, n_local - c);
-      for (int j = 0; j < cnt; ++j) {
+      return e_all;
+    };
+    auto ensure_wait = [&]() {
+      if (!waited) {
+        grid_dep_wait();
+        waited = true;
+      }
+    };
+    // stage and load the tokens held by lanes 0..cnt-1 of m, in lane order
+    auto issue = [&](const StageMeta &m, int cnt) {
+      for (int j = 0; j < cnt && !aborted; ++j) {
         StageMeta mj;
         mj.kv_base[0] = __shfl_sync(0xffffffffu, m.kv_base[0], j);
         mj.kv_base[1] = __shfl_sync(0xffffffffu, m.kv_base[1], j);
@@ -288,14 +313,15 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
         mj.pos[1] = __shfl_sync(0xffffffffu, m.pos[1], j);
         mj.ok[0] = __shfl_sync(0xffffffffu, m.ok[0], j);
         mj.ok[1] = __shfl_sync(0xffffffffu, m.ok[1], j);
-        const int ii = c + j;
-        const int s = ii % p.S;
+        mj.tok = __shfl_sync(0xffffffffu, m.tok, j);
+        mj.stop = 0;
+        const int s = issued % p.S;
         if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((ii / p.S) & 1) ^ 1, &s_abort)) {
+          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
             aborted = true;
           } else {
             meta[s] = mj;
-            const uint32_t tok = blockIdx.x + (uint32_t)ii * gridDim.x;
+            const uint32_t tok = (uint32_t)mj.tok;
             uint32_t tx = 0;
 #pragma unroll
             for (int k = 0; k < 2; ++k)
@@ -318,13 +344,48 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
                              (int64_t)mj.pos[k] * p.f_row_bytes,
                          (uint32_t)p.f_row_bytes, &full[s]);
             }
-            ++issued;
           }
         }
         aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
-        if (aborted) break;
+        if (!aborted) ++issued;
+      }
+    };
+    // the static share: tokens blockIdx.x + i * gridDim.x
+    for (int c = 0; c < n_static && !aborted; c += 32) {
+      StageMeta m;
+      const int i = c + lane;
+      const uint32_t e = resolve(i < n_static ? (int)blockIdx.x + i * (int)gridDim.x : -1, m);
+      ensure_wait();
+      raise(p.err, e);
+      issue(m, min(32, n_static - c));
+    }
+    // the claimed tail: the next claim is issued before the current chunk is staged
+    if (dyn) {
+      ensure_wait();
+      uint32_t next = 0;
+      if (lane == 0) next = atomicAdd(p.sched, (uint32_t)kDynChunk);
+      while (!aborted) {
+        const int64_t first = dyn0 + (int64_t)__shfl_sync(0xffffffffu, next, 0);
+        if (first >= p.T) break;
+        const int cnt = (int)min((int64_t)kDynChunk, (int64_t)p.T - first);
+        StageMeta m;
+        const uint32_t e = resolve(lane < cnt ? (int)first + lane : -1, m);
+        raise(p.err, e);
+        if (lane == 0) next = atomicAdd(p.sched, (uint32_t)kDynChunk);
+        issue(m, cnt);
       }
     }
+    // stop marker: the next stage carries no token
+    if (!aborted && lane == 0) {
+      const int s = issued % p.S;
+      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
+        aborted = true;
+      } else {
+        meta[s].stop = 1;
+        mbar_arrive(&full[s]);
+      }
+    }
+    aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
     if (aborted && lane == 0) {
       s_abort = 1;
       raise(p.err, ROPE_DEVERR_TIMEOUT);
@@ -337,14 +398,17 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
   } else if (warp == 1) {
     // -------------------------------------------------------------------- storer --
     if (lane == 0) {
-      for (int i = 0; i < n_local; ++i) {
+      int n_done = 0;  // tokens stored
+      for (int i = 0;; ++i) {
         const int s = i % p.S;
         if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort)) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);
           break;
         }
-        const uint32_t tok = blockIdx.x + (uint32_t)i * gridDim.x;
+        if (meta[s].stop) break;
+        n_done = i + 1;
+        const uint32_t tok = (uint32_t)meta[s].tok;
         const unsigned char *st = stages + (size_t)s * p.stage_bytes;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
@@ -379,7 +443,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
         }
       }
       bulk_wait_read<0>();
-      for (int i = max(0, n_local - kStoreLag); i < n_local; ++i) mbar_arrive(&empty[i % p.S]);
+      for (int i = max(0, n_done - kStoreLag); i < n_done; ++i) mbar_arrive(&empty[i % p.S]);
       bulk_wait<0>();
     }
   } else {
@@ -439,13 +503,18 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
     float fca[N], fsa[N], fcb[N], fsb[N];
     float ga[N], gb[N];
     int g_sel = -1;
-    for (int i = 0; i < n_local; ++i) {
+    for (int i = 0;; ++i) {
       const int s = i % p.S;
       if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
         if (lane == 0) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);
         }
+        break;
+      }
+      if (meta[s].stop) {  // hand the marker on to the storer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&done[s]);
         break;
       }
       unsigned char *st = stages + (size_t)s * p.stage_bytes;
@@ -558,6 +627,10 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&done[s]);
     }
+  }
+  if (p.sched != nullptr) {
+    __syncthreads();  // every claim of this CTA is made
+    if (tid == 0) sched_release(p.sched);
   }
 }
 

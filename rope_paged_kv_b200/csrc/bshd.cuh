@@ -4,7 +4,9 @@
 // keeps the dependency chain short instead of staging: one CTA per token, every thread
 // resolves the token's (valid, slot, position) itself from broadcast loads while its Q
 // loads are already in flight; K rows and the freqs row are then loaded in one round trip,
-// rotated, and stored.  No block-level barrier, no shared memory.
+// rotated, and stored.  No block-level barrier, no shared memory.  With launch overlap
+// mode 2 the descriptor loads come first, before the wait for the preceding kernels, and
+// the Q loads after it.
 #pragma once
 
 #include "common.cuh"
@@ -24,6 +26,7 @@ struct BshdParams {
   RopeDev rope;
   uint32_t *err;
   int32_t f_row_bytes;
+  int32_t overlap;  // launch-overlap mode (kOverlap*)
 };
 
 template <typename T, int D, int UQ, int UK>
@@ -36,14 +39,19 @@ __global__ void __launch_bounds__(kBshdThreads) bshd_rope_kernel(const __grid_co
   const int c0 = li * N;
   const bool in_rope = lane_in_rope(p.rope, c0);
   const int64_t n_tok = (int64_t)p.B * p.S;
+  const bool early_meta = p.overlap == kOverlapEarlyMeta;
+  if (tid == 0) grid_dep_launch_dependents();
+  if (!early_meta) grid_dep_wait();
   for (int64_t tok = blockIdx.x; tok < n_tok; tok += gridDim.x) {
     const T *qrow = reinterpret_cast<const T *>(p.q) + tok * p.n_q * D;
     T *orow = reinterpret_cast<T *>(p.out) + tok * p.n_q * D;
     uint4 vq[UQ];
+    if (!early_meta) {
 #pragma unroll
-    for (int u = 0; u < UQ; ++u) {
-      const int h = grp + u * G;
-      vq[u] = h < p.n_q ? ld_stream(qrow + (int64_t)h * D + c0) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < UQ; ++u) {
+        const int h = grp + u * G;
+        vq[u] = h < p.n_q ? ld_stream(qrow + (int64_t)h * D + c0) : make_uint4(0, 0, 0, 0);
+      }
     }
     const int b = (int)(tok / p.S), s = (int)(tok % p.S);
     const bool valid = (uint32_t)s < __ldg(p.valid + b);
@@ -55,6 +63,14 @@ __global__ void __launch_bounds__(kBshdThreads) bshd_rope_kernel(const __grid_co
         e = ROPE_DEVERR_BATCH;
       else if (pos >= p.rope.max_seq_len || pos >= p.cache_max_seq)
         e = ROPE_DEVERR_POSITION;
+    }
+    if (early_meta) {
+      grid_dep_wait();  // returns at once after the first token
+#pragma unroll
+      for (int u = 0; u < UQ; ++u) {
+        const int h = grp + u * G;
+        vq[u] = h < p.n_q ? ld_stream(qrow + (int64_t)h * D + c0) : make_uint4(0, 0, 0, 0);
+      }
     }
     if (tid == 0) raise(p.err, e);
     const bool ok = valid && e == 0;

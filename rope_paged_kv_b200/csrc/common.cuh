@@ -32,6 +32,40 @@ __device__ __forceinline__ void raise(uint32_t *err, uint32_t bits) {
   if (err != nullptr && bits != 0u) atomicOr(err, bits);
 }
 
+// Launch-overlap modes (rope_overlap_t): 0 plain launch; 1 programmatic dependent launch,
+// every global access after the predecessors completed; 2 the same, but descriptor arrays
+// (offsets, cache lengths, page and lookup tables, gammas) are read before that.
+constexpr int kOverlapOff = 0;
+constexpr int kOverlapPdl = 1;
+constexpr int kOverlapEarlyMeta = 2;
+
+// Token schedule of the staged kernels when the caller gives a workspace: a CTA first takes
+// its static share of the tokens, all but about kDynTail of them, then claims the rest
+// kDynChunk tokens at a time from a counter, so that CTAs that get more bandwidth take
+// more of the tail.
+constexpr int kDynTail = 4;
+constexpr int kDynChunk = 2;
+constexpr int kMaxStaticTokens = 32;
+
+// Tokens a CTA takes statically: all of its share without a workspace.
+__device__ __forceinline__ int static_tokens(int T, int n_local, bool dyn) {
+  if (!dyn) return n_local;
+  const int per = T / (int)gridDim.x;
+  return per > kDynTail ? min(per - kDynTail, kMaxStaticTokens) : 0;
+}
+
+// End of a CTA in a launch with a workspace (sched[0] the claim counter, sched[1] CTAs
+// finished): the last CTA to finish returns both words to zero for the next launch.
+// Called once per CTA, after the CTA's last claim.
+__device__ __forceinline__ void sched_release(uint32_t *sched) {
+  __threadfence();
+  if (atomicAdd(sched + 1, 1u) == gridDim.x - 1u) {
+    atomicExch(sched, 0u);
+    atomicExch(sched + 1, 0u);
+    __threadfence();
+  }
+}
+
 // sequence b with offs[b] <= row < offs[b+1] (offs a valid partition, row < offs[batch])
 __device__ __forceinline__ int find_seq(const uint32_t *offs, int batch, uint32_t row) {
   int lo = 0, hi = batch;

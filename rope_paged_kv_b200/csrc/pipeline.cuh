@@ -120,6 +120,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel of the stream (if
+// it was launched as a programmatic dependent) start its CTAs once every CTA here has
+// issued it; grid_dep_wait blocks until the kernels this one depends on have completed and
+// their writes are visible.  In a kernel not launched as a dependent, both do nothing.
+__device__ __forceinline__ void grid_dep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void st_shared_v4(void *p, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)), "r"(v.x),
                "r"(v.y), "r"(v.z), "r"(v.w)

@@ -1,8 +1,8 @@
 // radd.cuh -- in-place add of a [T, 2 * n_kv_heads * head_dim] tensor into the paged cache
-// (kv_cache_radd).  Same producer / consumer staging as the banded store: the producer
-// resolves each token's cache row (sequence + batch_offset, position, page translation) and
-// bulk-copies the token's input row together with the K and V cache rows it will add into;
-// the consumers add in float32, round once and store the rows back.
+// (kv_cache_radd).  Same producer / consumer staging and token schedule as the banded
+// store: the producer resolves each token's cache row (sequence + batch_offset, position,
+// page translation) and bulk-copies the token's input row together with the K and V cache
+// rows it will add into; the consumers add in float32, round once and store the rows back.
 #pragma once
 
 #include "banded.cuh"
@@ -23,11 +23,13 @@ struct RaddParams {
   uint32_t *err;
   int32_t S, stage_bytes, staged, kv_contig;  // kv_contig: a token's heads are adjacent
   int32_t bar_off, meta_off, offs_off;
+  int32_t overlap;  // launch-overlap mode (kOverlap*)
+  uint32_t *sched;  // claim counter + finished CTAs, or nullptr for a static schedule
 };
 
 struct RaddMeta {
   int64_t kv_base;
-  int32_t ok, pad;
+  int32_t ok, tok, stop, pad;
 };
 
 template <typename T, int D>
@@ -46,6 +48,7 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) grid_dep_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < p.S; ++s) {
       mbar_init(&full[s], 1);
@@ -54,6 +57,7 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
     s_abort = 0;
     fence_mbar_init();
   }
+  if (p.overlap != kOverlapEarlyMeta) grid_dep_wait();
   const bool good = stage_offsets(p.offs, p.batch, p.T, p.staged, s_offs);
   if (p.staged)
     for (int i = tid; i < p.batch; i += kRaddThreads) {
@@ -61,7 +65,11 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
       s_cl[i] = seq < p.cache.n_seqs ? __ldg(p.cache.cache_lengths + seq) : 0u;
     }
   if (!__syncthreads_and(good)) {
-    if (tid == 0) raise(p.err, ROPE_DEVERR_ROW_OFFSETS);
+    grid_dep_wait();
+    if (tid == 0) {
+      raise(p.err, ROPE_DEVERR_ROW_OFFSETS);
+      if (p.sched != nullptr) sched_release(p.sched);
+    }
     return;
   }
   const uint32_t *offs = p.staged ? s_offs : p.offs;
@@ -70,43 +78,51 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
   const uint32_t row_bytes = (uint32_t)(hidden * EB);  // one plane's heads of one token
 
   if (warp == 0) {
+    const bool dyn = p.sched != nullptr;
+    const int n_static = static_tokens(p.T, n_local, dyn);
+    const int dyn0 = n_static * (int)gridDim.x;  // first claimed token
     int issued = 0;
     bool aborted = false;
-    for (int c = 0; c < n_local && !aborted; c += 32) {
-      RaddMeta m{};
-      const int i = c + lane;
-      if (i < n_local) {
-        const uint32_t tok = blockIdx.x + (uint32_t)i * gridDim.x;
-        const int b = find_seq(offs, p.batch, tok);
-        const uint32_t t = tok - offs[b];
-        const uint64_t seq = (uint64_t)b + p.batch_offset;
-        uint32_t e = 0;
-        if (seq >= p.cache.n_seqs) {
-          e = ROPE_DEVERR_BATCH;
-        } else {
-          const uint32_t cl = p.staged ? s_cl[b] : __ldg(p.cache.cache_lengths + seq);
-          e = translate(p.cache, p.layer, seq, (uint64_t)cl + t, &m.kv_base);
-        }
-        m.ok = (e == 0);
-        raise(p.err, e);
+    bool waited = p.overlap != kOverlapEarlyMeta;
+    auto resolve = [&](int tok, RaddMeta &m) -> uint32_t {
+      m = RaddMeta{};
+      m.tok = tok;
+      if (tok < 0) return 0u;
+      const int b = find_seq(offs, p.batch, (uint32_t)tok);
+      const uint32_t t = (uint32_t)tok - offs[b];
+      const uint64_t seq = (uint64_t)b + p.batch_offset;
+      uint32_t e = 0;
+      if (seq >= p.cache.n_seqs) {
+        e = ROPE_DEVERR_BATCH;
+      } else {
+        const uint32_t cl = p.staged ? s_cl[b] : __ldg(p.cache.cache_lengths + seq);
+        e = translate(p.cache, p.layer, seq, (uint64_t)cl + t, &m.kv_base);
       }
-      const int cnt = min(32, n_local - c);
-      for (int j = 0; j < cnt; ++j) {
-        RaddMeta mj;
+      m.ok = (e == 0);
+      return e;
+    };
+    auto ensure_wait = [&]() {
+      if (!waited) {
+        grid_dep_wait();
+        waited = true;
+      }
+    };
+    auto issue = [&](const RaddMeta &m, int cnt) {
+      for (int j = 0; j < cnt && !aborted; ++j) {
+        RaddMeta mj{};
         mj.kv_base = __shfl_sync(0xffffffffu, m.kv_base, j);
         mj.ok = __shfl_sync(0xffffffffu, m.ok, j);
-        const int ii = c + j;
-        const int s = ii % p.S;
+        mj.tok = __shfl_sync(0xffffffffu, m.tok, j);
+        const int s = issued % p.S;
         if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((ii / p.S) & 1) ^ 1, &s_abort)) {
+          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
             aborted = true;
           } else {
             meta[s] = mj;
             mbar_arrive_expect_tx(&full[s], mj.ok ? 4u * row_bytes : 0u);
             if (mj.ok) {
-              const uint32_t tok = blockIdx.x + (uint32_t)ii * gridDim.x;
               unsigned char *st = smem + (size_t)s * p.stage_bytes;
-              bulk_g2s(st, reinterpret_cast<const unsigned char *>(p.a) + (int64_t)tok * p.a_stride * EB,
+              bulk_g2s(st, reinterpret_cast<const unsigned char *>(p.a) + (int64_t)mj.tok * p.a_stride * EB,
                        2u * row_bytes, &full[s]);
               const unsigned char *kb =
                   reinterpret_cast<const unsigned char *>(p.cache.k) + mj.kv_base * EB;
@@ -124,13 +140,45 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
                 }
               }
             }
-            ++issued;
           }
         }
         aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
-        if (aborted) break;
+        if (!aborted) ++issued;
+      }
+    };
+    for (int c = 0; c < n_static && !aborted; c += 32) {
+      RaddMeta m;
+      const int i = c + lane;
+      const uint32_t e = resolve(i < n_static ? (int)blockIdx.x + i * (int)gridDim.x : -1, m);
+      ensure_wait();
+      raise(p.err, e);
+      issue(m, min(32, n_static - c));
+    }
+    if (dyn) {
+      ensure_wait();
+      uint32_t next = 0;
+      if (lane == 0) next = atomicAdd(p.sched, (uint32_t)kDynChunk);
+      while (!aborted) {
+        const int64_t first = dyn0 + (int64_t)__shfl_sync(0xffffffffu, next, 0);
+        if (first >= p.T) break;
+        const int cnt = (int)min((int64_t)kDynChunk, (int64_t)p.T - first);
+        RaddMeta m;
+        const uint32_t e = resolve(lane < cnt ? (int)first + lane : -1, m);
+        raise(p.err, e);
+        if (lane == 0) next = atomicAdd(p.sched, (uint32_t)kDynChunk);
+        issue(m, cnt);
       }
     }
+    if (!aborted && lane == 0) {  // stop marker
+      const int s = issued % p.S;
+      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
+        aborted = true;
+      } else {
+        meta[s].stop = 1;
+        mbar_arrive(&full[s]);
+      }
+    }
+    aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
     if (aborted && lane == 0) {
       s_abort = 1;
       raise(p.err, ROPE_DEVERR_TIMEOUT);
@@ -143,7 +191,7 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
     const int ctid = tid - 32;
     const int li = ctid % L, grp = ctid / L;
     const int rows = 2 * p.n_kv;
-    for (int i = 0; i < n_local; ++i) {
+    for (int i = 0;; ++i) {
       const int s = i % p.S;
       if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
         if (lane == 0) {
@@ -153,6 +201,7 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
         break;
       }
       const RaddMeta m = meta[s];
+      if (m.stop) break;
       if (m.ok) {
         const unsigned char *st = smem + (size_t)s * p.stage_bytes;
         for (int j = grp; j < rows; j += G) {
@@ -171,6 +220,10 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
+  }
+  if (p.sched != nullptr) {
+    __syncthreads();  // every claim of this CTA is made
+    if (tid == 0) sched_release(p.sched);
   }
 }
 

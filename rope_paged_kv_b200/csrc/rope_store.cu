@@ -13,6 +13,7 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <type_traits>
 
 namespace rs {
@@ -39,6 +40,34 @@ static BandedShape pick_shape(const BandedParams &p, bool norm) {
 }
 
 // ------------------------------------------------------------------------ host side --
+
+// launch-overlap mode of every launch that follows (rope_set_launch_overlap)
+static std::atomic<int> g_overlap{kOverlapPdl};
+
+// Launch `kern` with one parameter block; modes 1 and 2 launch it as a programmatic
+// dependent of the previous kernel in the stream.
+template <typename K, typename P>
+static rope_status_t launch(K kern, int grid, int threads, size_t smem, cudaStream_t st,
+                            const P &p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (p.overlap != kOverlapOff) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return ROPE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? ROPE_OK : ROPE_ERR_CUDA;
+}
+
+static bool sched_ok(const uint32_t *sched) {
+  return (reinterpret_cast<uintptr_t>(sched) & 3u) == 0;
+}
 
 static int sm_count() {
   static int cached[64] = {0};
@@ -268,8 +297,7 @@ static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStr
   if (occ <= 0) return ROPE_ERR_UNSUPPORTED;  // the stage ring does not fit
   const int64_t slots = (int64_t)sm_count() * occ;
   const int grid = (int)(slots < p.T ? slots : p.T);
-  kern<<<grid, pipe_threads<CW>(), smem, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ROPE_OK : ROPE_ERR_CUDA;
+  return launch(kern, grid, pipe_threads<CW>(), smem, st, p);
 }
 
 template <typename T, int D, bool NORM>
@@ -315,10 +343,8 @@ static rope_status_t launch_bshd_t(const BshdParams &p, cudaStream_t st) {
   const int64_t cap = (int64_t)1 << 30;
   const int grid = (int)(n_tok < cap ? n_tok : cap);
   if (p.n_q <= 2 * G && p.n_kv <= G)
-    bshd_rope_kernel<T, D, 2, 1><<<grid, kBshdThreads, 0, st>>>(p);
-  else
-    bshd_rope_kernel<T, D, 4, 2><<<grid, kBshdThreads, 0, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ROPE_OK : ROPE_ERR_CUDA;
+    return launch(bshd_rope_kernel<T, D, 2, 1>, grid, kBshdThreads, 0, st, p);
+  return launch(bshd_rope_kernel<T, D, 4, 2>, grid, kBshdThreads, 0, st, p);
 }
 
 template <typename T>
@@ -357,8 +383,7 @@ static rope_status_t launch_radd_t(const RaddParams &p, size_t smem, cudaStream_
   if (occ <= 0) return ROPE_ERR_UNSUPPORTED;
   const int64_t slots = (int64_t)sm_count() * occ;
   const int grid = (int)(slots < p.T ? slots : p.T);
-  kern<<<grid, kRaddThreads, smem, st>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ROPE_OK : ROPE_ERR_CUDA;
+  return launch(kern, grid, kRaddThreads, smem, st, p);
 }
 
 template <typename T>
@@ -392,9 +417,10 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
                                             const rope_freqs_t *freqs,
                                             const rope_paged_cache_t *kv, uint32_t layer_idx,
                                             void *q_out, int64_t q_out_row_stride,
-                                            uint32_t *err_word, rope_stream_t stream) {
+                                            uint32_t *err_word, uint32_t *sched,
+                                            rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
-  if (kv == nullptr) return ROPE_ERR_INVALID_ARG;
+  if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
   const int dtype = kv->dtype, D = kv->head_dim;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
@@ -413,6 +439,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
   p.T = total_tokens;
   p.layer = layer_idx;
   p.err = err_word;
+  p.sched = sched;
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
   if (p.work_total + Hk == 0) return ROPE_OK;
   return launch_banded(dtype, D, false, p, (cudaStream_t)stream);
 }
@@ -426,9 +454,9 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
                                           float weight_offset, int32_t multiply_before_cast,
                                           uint32_t layer_idx, void *q_out,
                                           int64_t q_out_row_stride, uint32_t *err_word,
-                                          rope_stream_t stream) {
+                                          uint32_t *sched, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
-  if (kv == nullptr) return ROPE_ERR_INVALID_ARG;
+  if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
   const int dtype = kv->dtype, D = kv->head_dim;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
@@ -448,6 +476,8 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
   p.T = total_tokens;
   p.layer = layer_idx;
   p.err = err_word;
+  p.sched = sched;
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
   p.weight_offset = round_to_elem(weight_offset, dtype);
   if (p.work_total + Hk == 0) return ROPE_OK;
   return launch_banded(dtype, D, true, p, (cudaStream_t)stream);
@@ -459,10 +489,11 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
                                                int32_t batch, int32_t total_tokens,
                                                const rope_freqs_t *freqs, float weight_offset,
                                                int32_t multiply_before_cast, uint32_t layer_idx,
-                                               uint32_t *err_word, rope_stream_t stream) {
+                                               uint32_t *err_word, uint32_t *sched,
+                                               rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
   if (main_band == nullptr || index_band == nullptr || main_band->cache == nullptr ||
-      index_band->cache == nullptr)
+      index_band->cache == nullptr || !sched_ok(sched))
     return ROPE_ERR_INVALID_ARG;
   const rope_paged_cache_t *mc = main_band->cache, *ic = index_band->cache;
   // the rope geometry must agree across the bands
@@ -493,6 +524,8 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
   p.T = total_tokens;
   p.layer = layer_idx;
   p.err = err_word;
+  p.sched = sched;
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
   p.weight_offset = round_to_elem(weight_offset, dtype);
   if (p.work_total == 0) return ROPE_OK;
   return launch_banded(dtype, D, true, p, (cudaStream_t)stream);
@@ -540,6 +573,7 @@ rope_status_t qk_rope_bshd_continuous(const void *q_proj, int32_t batch, int32_t
   p.layer = layer_idx;
   p.err = err_word;
   p.f_row_bytes = p.rope.R * (p.rope.dtype == 2 ? 4 : 2);
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == ROPE_DTYPE_BF16) return launch_bshd_d<__nv_bfloat16>(D, p, st);
   if (dtype == ROPE_DTYPE_F16) return launch_bshd_d<__half>(D, p, st);
@@ -549,9 +583,9 @@ rope_status_t qk_rope_bshd_continuous(const void *q_proj, int32_t batch, int32_t
 rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_tokens,
                             const rope_paged_cache_t *kv, const uint32_t *input_row_offsets,
                             int32_t batch, uint32_t batch_offset, uint32_t layer_idx,
-                            uint32_t *err_word, rope_stream_t stream) {
+                            uint32_t *err_word, uint32_t *sched, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
-  if (kv == nullptr || a == nullptr) return ROPE_ERR_INVALID_ARG;
+  if (kv == nullptr || a == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
   const int dtype = kv->dtype, D = kv->head_dim;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
@@ -572,6 +606,8 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
   p.batch_offset = batch_offset;
   p.layer = layer_idx;
   p.err = err_word;
+  p.sched = sched;
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
   p.kv_contig = kv->head_stride == D ? 1 : 0;
   const size_t smem = layout_radd(p, D, eb);
   if (smem > 227 * 1024) return ROPE_ERR_UNSUPPORTED;
@@ -580,5 +616,14 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
   if (dtype == ROPE_DTYPE_F16) return launch_radd_d<__half>(D, p, smem, st);
   return launch_radd_d<float>(D, p, smem, st);
 }
+
+rope_status_t rope_set_launch_overlap(int32_t mode) {
+  if (mode != ROPE_OVERLAP_OFF && mode != ROPE_OVERLAP_PDL && mode != ROPE_OVERLAP_PDL_EARLY_METADATA)
+    return ROPE_ERR_INVALID_ARG;
+  g_overlap.store(mode, std::memory_order_relaxed);
+  return ROPE_OK;
+}
+
+int32_t rope_get_launch_overlap(void) { return g_overlap.load(std::memory_order_relaxed); }
 
 }  // extern "C"

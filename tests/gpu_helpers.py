@@ -46,6 +46,19 @@ def err_word() -> torch.Tensor:
     return torch.zeros(1, dtype=torch.int32, device=DEV)
 
 
+# The staged entry points run with a scheduling workspace (the claimed-tail token schedule)
+# unless a test switches this off to get the static schedule.
+USE_SCHED = True
+
+
+def sched_of(s) -> torch.Tensor | None:
+    if not USE_SCHED:
+        return None
+    if getattr(s, "sched", None) is None:
+        s.sched = rs.sched_workspace(DEV)
+    return s.sched
+
+
 class Staged:
     """A workload's tensors on the device, with the binding's descriptors."""
 
@@ -67,11 +80,11 @@ def stage_ragged(w: W.RaggedStore) -> Staged:
 def launch_ragged(w: W.RaggedStore, s: Staged, stream=None) -> None:
     if w.q_gamma is None:
         rs.rope_split_store_paged_ragged(s.qkv, w.n_q_heads, s.offs, s.freqs, s.kv,
-                                         w.layer_idx, s.q_out, s.err, stream)
+                                         w.layer_idx, s.q_out, s.err, stream, sched_of(s))
     else:
         rs.fused_qk_rmsnorm_rope_paged(s.qkv, w.n_q_heads, s.offs, s.freqs, s.kv, s.q_gamma,
                                        s.k_gamma, w.epsilon, w.weight_offset, w.layer_idx,
-                                       s.q_out, True, s.err, stream)
+                                       s.q_out, True, s.err, stream, sched_of(s))
 
 
 def run_ragged(w: W.RaggedStore):
@@ -102,7 +115,8 @@ def stage_dual(w: W.DualBand) -> Staged:
 
 def launch_dual(w: W.DualBand, s: Staged, stream=None) -> None:
     rs.fused_dual_qk_rmsnorm_rope_paged(s.main, s.index, s.offs, w.total_tokens, s.freqs,
-                                        w.weight_offset, w.layer_idx, True, s.err, stream)
+                                        w.weight_offset, w.layer_idx, True, s.err, stream,
+                                        sched_of(s))
 
 
 def run_dual(w: W.DualBand):
@@ -146,7 +160,8 @@ def stage_radd(w: W.Radd) -> Staged:
 
 
 def launch_radd(w: W.Radd, s: Staged, stream=None) -> None:
-    rs.kv_cache_radd(s.a, s.kv, s.offs, w.batch_offset, w.layer_idx, s.err, stream)
+    rs.kv_cache_radd(s.a, s.kv, s.offs, w.batch_offset, w.layer_idx, s.err, stream,
+                     sched_of(s))
 
 
 def run_radd(w: W.Radd):

@@ -20,14 +20,15 @@ def rs():
 
 def _declared():
     text = open(os.path.join(ROOT, "include", "rope_store.h")).read()
-    return re.findall(r"^(?:rope_status_t|const char \*)\s*(\w+)\(", text, re.M)
+    return re.findall(r"^(?:rope_status_t|int32_t|const char \*)\s*(\w+)\(", text, re.M)
 
 
 def test_header_declares_the_entry_points():
     names = set(_declared())
     assert {"rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
             "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous",
-            "kv_cache_radd", "rope_status_string"} <= names
+            "kv_cache_radd", "rope_status_string", "rope_set_launch_overlap",
+            "rope_get_launch_overlap"} <= names
 
 
 def test_library_exports_every_declared_symbol(rs):
@@ -76,42 +77,42 @@ def test_host_argument_checks_need_no_gpu(rs):
                           fake, 2)
     call = lib.rope_split_store_paged_ragged
     # NULL descriptors / pointers
-    assert call(fake, 512, 8, 4, fake, 2, None, ctypes.byref(kv), 1, fake, 256, None,
+    assert call(fake, 512, 8, 4, fake, 2, None, ctypes.byref(kv), 1, fake, 256, None, None,
                 None) == rs.ERR_INVALID_ARG
     assert call(fake, 512, 8, 4, None, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.ERR_INVALID_ARG
+                None, None, None) == rs.ERR_INVALID_ARG
     # layer past num_layers
     assert call(fake, 512, 8, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 2, fake, 256,
-                None, None) == rs.ERR_INVALID_ARG
+                None, None, None) == rs.ERR_INVALID_ARG
     # odd rope_dim, rope_dim > head_dim
     for bad in (rs.c_freqs(fake, 2, 64, 63, 1, -1), rs.c_freqs(fake, 2, 64, 66, 1, -1)):
         assert call(fake, 512, 8, 4, fake, 2, ctypes.byref(bad), ctypes.byref(kv), 1, fake,
-                    256, None, None) == rs.ERR_INVALID_ARG
+                    256, None, None, None) == rs.ERR_INVALID_ARG
     # half-split pairs that straddle a 16-byte vector
     bad = rs.c_freqs(fake, 2, 64, 8, 0, -1)
     assert call(fake, 512, 8, 4, fake, 2, ctypes.byref(bad), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.ERR_UNSUPPORTED
+                None, None, None) == rs.ERR_UNSUPPORTED
     # unsupported head_dim, misaligned row stride, misaligned base
     kv96 = rs.c_paged_cache(fake, fake, 0, 2, 96, 16, 8, 2, 4096, 2048, 192, 96, fake, 4, 4,
                             fake, 2)
     assert call(fake, 768, 8, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv96), 1, fake, 384,
-                None, None) == rs.ERR_UNSUPPORTED
+                None, None, None) == rs.ERR_UNSUPPORTED
     assert call(fake, 515, 8, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.ERR_UNSUPPORTED
+                None, None, None) == rs.ERR_UNSUPPORTED
     assert call(fake + 2, 512, 8, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.ERR_UNSUPPORTED
+                None, None, None) == rs.ERR_UNSUPPORTED
     # more sequences than the cache describes; tokens without sequences
     assert call(fake, 512, 8, 4, fake, 3, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.ERR_INVALID_ARG
+                None, None, None) == rs.ERR_INVALID_ARG
     assert call(fake, 512, 8, 4, fake, 0, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.ERR_INVALID_ARG
+                None, None, None) == rs.ERR_INVALID_ARG
     # empty work: OK without a launch
     assert call(fake, 512, 0, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
-                None, None) == rs.OK
+                None, None, None) == rs.OK
     # multiply_before_cast = 0 is not built
     assert lib.fused_qk_rmsnorm_rope_paged(fake, 512, 8, 4, fake, 2, ctypes.byref(f),
                                            ctypes.byref(kv), fake, fake, 1e-6, 0.0, 0, 1, fake,
-                                           256, None, None) == rs.ERR_UNSUPPORTED
+                                           256, None, None, None) == rs.ERR_UNSUPPORTED
     # dual band: geometry must agree across bands
     kv128 = rs.c_paged_cache(fake, None, 0, 1, 128, 16, 8, 2, 4096, 2048, 128, 128, fake, 4,
                              4, fake, 2)
@@ -120,14 +121,35 @@ def test_host_argument_checks_need_no_gpu(rs):
     ib = rs.c_norm_band(fake, 1024, 512, 768, -1, 1, ctypes.pointer(kv128), fake, fake, 1e-6,
                         fake, 128)
     assert lib.fused_dual_qk_rmsnorm_rope_paged(ctypes.byref(mb), ctypes.byref(ib), fake, 2, 8,
-                                                ctypes.byref(f), 0.0, 1, 1, None,
+                                                ctypes.byref(f), 0.0, 1, 1, None, None,
                                                 None) == rs.ERR_INVALID_ARG
     # radd needs a V plane
     kvk = rs.c_paged_cache(fake, None, 0, 2, 64, 16, 8, 2, 4096, 2048, 128, 64, fake, 4, 4,
                            fake, 2)
-    assert lib.kv_cache_radd(fake, 256, 8, ctypes.byref(kvk), fake, 2, 0, 1, None,
+    assert lib.kv_cache_radd(fake, 256, 8, ctypes.byref(kvk), fake, 2, 0, 1, None, None,
                              None) == rs.ERR_INVALID_ARG
     # BSHD: head_dim must match the cache
     cc = rs.c_cont_cache(fake, None, 0, 2, 64, 4, 1, 64, 8192, 8192, 128, 64, fake, fake, 4)
     assert lib.qk_rope_bshd_continuous(fake, 2, 1, 4, 128, ctypes.byref(cc), ctypes.byref(f),
                                        0, fake, fake, None, None) == rs.ERR_INVALID_ARG
+
+    # a scheduling workspace must hold aligned uint32 words
+    assert call(fake, 512, 8, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
+                None, fake + 2, None) == rs.ERR_INVALID_ARG
+    assert lib.kv_cache_radd(fake, 256, 8, ctypes.byref(kvk), fake, 2, 0, 1, None, fake + 1,
+                             None) == rs.ERR_INVALID_ARG
+
+
+def test_launch_overlap_mode(rs):
+    lib = rs.raw_library()
+    before = lib.rope_get_launch_overlap()
+    assert before == rs.OVERLAP_PDL  # the default
+    try:
+        for mode in (rs.OVERLAP_OFF, rs.OVERLAP_PDL_EARLY_METADATA, rs.OVERLAP_PDL):
+            assert lib.rope_set_launch_overlap(mode) == rs.OK
+            assert lib.rope_get_launch_overlap() == mode
+        assert lib.rope_set_launch_overlap(3) == rs.ERR_INVALID_ARG
+        assert lib.rope_set_launch_overlap(-1) == rs.ERR_INVALID_ARG
+        assert lib.rope_get_launch_overlap() == rs.OVERLAP_PDL
+    finally:
+        lib.rope_set_launch_overlap(before)
