@@ -260,6 +260,28 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
                             int32_t batch, uint32_t batch_offset, uint32_t layer_idx,
                             uint32_t *err_word, uint32_t *sched, rope_stream_t stream);
 
+/* rope_split_store_paged_ragged_noalloc -- rope_split_store_paged_ragged with the
+ * claimed-tail schedule, for callers that cannot allocate device memory: for example a
+ * plug-in inside an engine that hands out all device memory from its own pool and allows no
+ * other allocation, or code on a latency-critical path that must not call cudaMalloc or
+ * cudaFree (either may synchronise the device).  The pages have no counterpart of this
+ * call; it is a launch variant, not a different operation.
+ * Arguments and results are those of rope_split_store_paged_ragged without `sched`: the
+ * scheduling workspace is a 256-byte array inside the library, one per device, of which the
+ * schedule uses ROPE_SCHED_WORDS words whatever the call's sizes (so no size is too large
+ * for it).  The call allocates nothing; it clears those words on `stream` before its
+ * launch.  The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  Every call on a device
+ * shares the array, so calls that can overlap on the GPU (different streams) race on it and
+ * may skip tokens: keep the calls of this entry point in one stream, or use
+ * rope_split_store_paged_ragged with a workspace per stream.  ROPE_ERR_CUDA if the lookup
+ * or the clearing fails. */
+rope_status_t rope_split_store_paged_ragged_noalloc(
+    const void *qkv, int64_t qkv_row_stride, int32_t total_tokens, int32_t n_q_heads,
+    const uint32_t *input_row_offsets, int32_t batch, const rope_freqs_t *freqs,
+    const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
+    uint32_t *err_word, rope_stream_t stream);
+
 /* A static, human-readable name of a status code. */
 const char *rope_status_string(rope_status_t status);
 

@@ -101,12 +101,15 @@ _lib.qk_rope_bshd_continuous.argtypes = [
     _vp, _i32, _i32, _i32, _i32, _P(c_cont_cache), _P(c_freqs), _u32, _vp, _vp, _vp, _vp]
 _lib.kv_cache_radd.argtypes = [
     _vp, _i64, _i32, _P(c_paged_cache), _vp, _i32, _u32, _u32, _vp, _vp, _vp]
+_lib.rope_split_store_paged_ragged_noalloc.argtypes = [
+    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp,
+    _vp]
 _lib.rope_set_launch_overlap.argtypes = [_i32]
 _lib.rope_get_launch_overlap.argtypes = []
 _lib.rope_get_launch_overlap.restype = _i32
 for _f in ("rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
            "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd",
-           "rope_set_launch_overlap"):
+           "rope_set_launch_overlap", "rope_split_store_paged_ragged_noalloc"):
     getattr(_lib, _f).restype = ctypes.c_int
 _lib.rope_status_string.argtypes = [ctypes.c_int]
 _lib.rope_status_string.restype = ctypes.c_char_p
@@ -278,6 +281,21 @@ def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, freqs: Freq
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
         _row_stride(q_out), _ptr(err_word), _sched(sched), _stream(stream)),
         "rope_split_store_paged_ragged")
+
+
+def rope_split_store_paged_ragged_noalloc(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
+                                          kv: PagedCache, layer_idx, q_out, err_word=None,
+                                          stream=None) -> None:
+    """rope_split_store_paged_ragged for callers that cannot allocate device memory: the
+    scheduling workspace is the library's own per-device array (calls on different streams
+    must not overlap)."""
+    offs = _idx(input_row_offsets)
+    f, c = freqs.c(), kv.c()
+    _check(_lib.rope_split_store_paged_ragged_noalloc(
+        qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
+        offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
+        _row_stride(q_out), _ptr(err_word), _stream(stream)),
+        "rope_split_store_paged_ragged_noalloc")
 
 
 def fused_qk_rmsnorm_rope_paged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,

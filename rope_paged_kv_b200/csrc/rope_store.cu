@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 #include <type_traits>
 
 namespace rs {
@@ -395,6 +396,33 @@ static rope_status_t launch_radd_d(int D, const RaddParams &p, size_t smem, cuda
   return ROPE_ERR_UNSUPPORTED;
 }
 
+// ------------------------------------------------------- allocation-free entry point --
+// Scheduling workspace of rope_split_store_paged_ragged_noalloc.  Every device that loads
+// the library holds one copy of this array until the process exits, and every call of that
+// entry point on the device uses it.  The schedule needs ROPE_SCHED_WORDS words of it
+// whatever the call's sizes.
+constexpr int kNoAllocScratchWords = 64;  // 256 bytes
+static_assert(ROPE_SCHED_WORDS <= kNoAllocScratchWords, "the schedule must fit the array");
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchWords];
+
+// The array's device address on the current device.  In host code the symbol only names a
+// host-side stand-in, so the address is looked up once per device, with that device
+// current, and cached; nullptr if the lookup fails.
+static uint32_t *noalloc_scratch() {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static uint32_t *addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint32_t *>(p);
+  }
+  return addr[dev];
+}
+
 }  // namespace rs
 
 using namespace rs;
@@ -615,6 +643,23 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
   if (dtype == ROPE_DTYPE_BF16) return launch_radd_d<__nv_bfloat16>(D, p, smem, st);
   if (dtype == ROPE_DTYPE_F16) return launch_radd_d<__half>(D, p, smem, st);
   return launch_radd_d<float>(D, p, smem, st);
+}
+
+rope_status_t rope_split_store_paged_ragged_noalloc(
+    const void *qkv, int64_t qkv_row_stride, int32_t total_tokens, int32_t n_q_heads,
+    const uint32_t *input_row_offsets, int32_t batch, const rope_freqs_t *freqs,
+    const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
+    uint32_t *err_word, rope_stream_t stream) {
+  if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
+  uint32_t *scratch = noalloc_scratch();
+  if (scratch == nullptr) return ROPE_ERR_CUDA;
+  // the workspace starts each call at zero (a call that gave up early may have left counts)
+  if (cudaMemsetAsync(scratch, 0, ROPE_SCHED_WORDS * sizeof(uint32_t), (cudaStream_t)stream) !=
+      cudaSuccess)
+    return ROPE_ERR_CUDA;
+  return rope_split_store_paged_ragged(qkv, qkv_row_stride, total_tokens, n_q_heads,
+                                       input_row_offsets, batch, freqs, kv, layer_idx, q_out,
+                                       q_out_row_stride, err_word, scratch, stream);
 }
 
 rope_status_t rope_set_launch_overlap(int32_t mode) {
