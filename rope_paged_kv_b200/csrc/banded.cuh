@@ -201,8 +201,16 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
   }
 }
 
+#ifndef ROPE_LIGHT_MIN_CTAS
+#define ROPE_LIGHT_MIN_CTAS 2
+#endif
+// resident CTAs per SM the register budget is sized for: the light shape (<= 4 consumer
+// warps) and the heavy one
+template <int CW>
+__host__ __device__ constexpr int pipe_min_ctas() { return CW <= 4 ? ROPE_LIGHT_MIN_CTAS : 2; }
+
 template <typename T, int D, bool NORM, int CW, int LAG>
-__global__ void __launch_bounds__(pipe_threads<CW>(), 2)
+__global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     banded_store_kernel(const __grid_constant__ BandedParams p) {
   constexpr int kConsumerWarps = CW;
   constexpr int kConsumers = 32 * CW;

@@ -2,16 +2,17 @@
 // (kv_cache_radd).  Same producer / consumer staging and token schedule as the banded
 // store: the producer resolves each token's cache row (sequence + batch_offset, position,
 // page translation) and bulk-copies the token's input row together with the K and V cache
-// rows it will add into; the consumers add in float32, round once and store the rows back.
+// rows it will add into; the consumers add in float32, round once and write the sums over
+// the staged cache rows; the storer warp bulk-copies those rows back to the cache.
 #pragma once
 
 #include "banded.cuh"
 
 namespace rs {
 
-constexpr int kRaddConsumerWarps = 8;
-constexpr int kRaddConsumers = 32 * kRaddConsumerWarps;
-constexpr int kRaddThreads = kRaddConsumers + 32;  // + producer warp
+// CW consumer warps + the producer and storer warps
+template <int CW>
+__host__ __device__ constexpr int radd_threads() { return 32 * (CW + 2); }
 
 struct RaddParams {
   const void *a;
@@ -32,16 +33,19 @@ struct RaddMeta {
   int32_t ok, tok, stop, pad;
 };
 
-template <typename T, int D>
-__global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_constant__ RaddParams p) {
+template <typename T, int D, int CW, int LAG>
+__global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __grid_constant__ RaddParams p) {
   using VT = Vec<T>;
   constexpr int N = VT::N;
   constexpr int L = D / N;
-  constexpr int G = kRaddConsumers / L;
+  constexpr int kConsumers = 32 * CW;
+  constexpr int kThreads = radd_threads<CW>();
+  constexpr int G = kConsumers / L;
   constexpr int EB = (int)sizeof(T);
   extern __shared__ __align__(128) unsigned char smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + p.bar_off);
-  uint64_t *empty = full + p.S;
+  uint64_t *done = full + p.S;
+  uint64_t *empty = done + p.S;
   RaddMeta *meta = reinterpret_cast<RaddMeta *>(smem + p.meta_off);
   uint32_t *s_offs = reinterpret_cast<uint32_t *>(smem + p.offs_off);
   uint32_t *s_cl = s_offs + (p.batch + 1);
@@ -52,7 +56,8 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
   if (tid == 0) {
     for (int s = 0; s < p.S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kRaddConsumerWarps);
+      mbar_init(&done[s], CW);
+      mbar_init(&empty[s], 1);
     }
     s_abort = 0;
     fence_mbar_init();
@@ -60,7 +65,7 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
   if (p.overlap != kOverlapEarlyMeta) grid_dep_wait();
   const bool good = stage_offsets(p.offs, p.batch, p.T, p.staged, s_offs);
   if (p.staged)
-    for (int i = tid; i < p.batch; i += kRaddThreads) {
+    for (int i = tid; i < p.batch; i += kThreads) {
       const uint64_t seq = (uint64_t)i + p.batch_offset;
       s_cl[i] = seq < p.cache.n_seqs ? __ldg(p.cache.cache_lengths + seq) : 0u;
     }
@@ -187,8 +192,47 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
         mbar_wait(&full[ii % p.S], (ii / p.S) & 1, &never);
       }
     }
+  } else if (warp == 1) {
+    // storer: the summed K and V rows back to the cache, LAG bulk groups kept in flight
+    if (lane == 0) {
+      int n_done = 0;
+      for (int i = 0;; ++i) {
+        const int s = i % p.S;
+        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort)) {
+          s_abort = 1;
+          raise(p.err, ROPE_DEVERR_TIMEOUT);
+          break;
+        }
+        if (meta[s].stop) break;
+        n_done = i + 1;
+        if (meta[s].ok) {
+          const unsigned char *st = smem + (size_t)s * p.stage_bytes;
+          const int64_t base = meta[s].kv_base;
+          for (int plane = 0; plane < 2; ++plane) {
+            unsigned char *dst =
+                reinterpret_cast<unsigned char *>(plane ? p.cache.v : p.cache.k) + base * EB;
+            const unsigned char *src = st + (2 + plane) * row_bytes;
+            if (p.kv_contig) {
+              bulk_s2g(dst, src, row_bytes);
+            } else {
+              for (int h = 0; h < p.n_kv; ++h)
+                bulk_s2g(dst + (int64_t)h * p.cache.head_stride * EB, src + h * D * EB,
+                         (uint32_t)(D * EB));
+            }
+          }
+        }
+        bulk_commit();
+        if (i >= LAG) {
+          bulk_wait_read<LAG>();
+          mbar_arrive(&empty[(i - LAG) % p.S]);
+        }
+      }
+      bulk_wait_read<0>();
+      for (int i = max(0, n_done - LAG); i < n_done; ++i) mbar_arrive(&empty[i % p.S]);
+      bulk_wait<0>();
+    }
   } else {
-    const int ctid = tid - 32;
+    const int ctid = tid - 64;
     const int li = ctid % L, grp = ctid / L;
     const int rows = 2 * p.n_kv;
     for (int i = 0;; ++i) {
@@ -201,9 +245,8 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
         break;
       }
       const RaddMeta m = meta[s];
-      if (m.stop) break;
-      if (m.ok) {
-        const unsigned char *st = smem + (size_t)s * p.stage_bytes;
+      if (!m.stop && m.ok) {
+        unsigned char *st = smem + (size_t)s * p.stage_bytes;
         for (int j = grp; j < rows; j += G) {
           const int plane = j >= p.n_kv ? 1 : 0, h = j - plane * p.n_kv;
           const int64_t e0 = (int64_t)plane * hidden + (int64_t)h * D + li * N;
@@ -212,13 +255,13 @@ __global__ void __launch_bounds__(kRaddThreads, 1) radd_kernel(const __grid_cons
           VT::widen(ld_shared_v4(st + 2 * row_bytes + e0 * EB), xc);
 #pragma unroll
           for (int e = 0; e < N; ++e) xc[e] = xc[e] + xa[e];
-          T *dst = reinterpret_cast<T *>(plane ? p.cache.v : p.cache.k) + m.kv_base +
-                   (int64_t)h * p.cache.head_stride + li * N;
-          st_plain(dst, VT::narrow(xc));
+          st_shared_v4(st + 2 * row_bytes + e0 * EB, VT::narrow(xc));
         }
+        fence_proxy_async_smem();  // the storer's bulk copies read the sums
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+      if (lane == 0) mbar_arrive(&done[s]);  // the stop marker is handed on too
+      if (m.stop) break;
     }
   }
   if (p.sched != nullptr) {

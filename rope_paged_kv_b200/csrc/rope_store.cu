@@ -34,10 +34,27 @@ struct BandedShape {
 #endif
 // <= 64 Q+K head rows a token, no norm
 constexpr BandedShape kLightShape = {ROPE_LIGHT_CW, ROPE_LIGHT_LAG, ROPE_LIGHT_RING};
-constexpr BandedShape kHeavyShape = {8, 0, 96};  // RMSNorm or many heads
+// RMSNorm or many heads: six or eight consumer warps, whichever takes fewer passes over a
+// token's head rows (six on a tie: 116.6 vs 119.9 us on the per-head-norm workload, whose
+// 72 rows take three passes either way; eight on the dual-band one, 81 rows in three
+// passes instead of four: 248.4 vs 264.8 us)
+constexpr BandedShape kMidShape = {6, 0, 96};
+constexpr BandedShape kHeavyShape = {8, 0, 96};
 
-static BandedShape pick_shape(const BandedParams &p, bool norm) {
-  return (!norm && p.work_total <= 64) ? kLightShape : kHeavyShape;
+enum ShapeId { kLight = 0, kMid = 1, kHeavy = 2 };
+
+static int passes(const BandedParams &p, int D, int cw) {
+  const int rows_per_pass = 32 * cw / (D / (2 * (16 / p.elem_bytes)));
+  return (p.work_total + rows_per_pass - 1) / rows_per_pass;
+}
+
+static ShapeId pick_shape(const BandedParams &p, int D, bool norm) {
+  if (!norm && p.work_total <= 64) return kLight;
+  return passes(p, D, kMidShape.cw) <= passes(p, D, kHeavyShape.cw) ? kMid : kHeavy;
+}
+
+static const BandedShape &shape_of(ShapeId id) {
+  return id == kLight ? kLightShape : id == kMid ? kMidShape : kHeavyShape;
 }
 
 // ------------------------------------------------------------------------ host side --
@@ -302,38 +319,39 @@ static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStr
 }
 
 template <typename T, int D, bool NORM>
-static rope_status_t launch_banded_s(const BandedShape &sh, const BandedParams &p, size_t smem,
+static rope_status_t launch_banded_s(ShapeId id, const BandedParams &p, size_t smem,
                                      cudaStream_t st) {
-  if (sh.cw == kLightShape.cw)
+  if (id == kLight)
     return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
+  if (id == kMid) return launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag>(p, smem, st);
   return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag>(p, smem, st);
 }
 
 template <typename T, bool NORM>
-static rope_status_t launch_banded_d(int D, const BandedShape &sh, const BandedParams &p,
-                                     size_t smem, cudaStream_t st) {
-  if (D == 64) return launch_banded_s<T, 64, NORM>(sh, p, smem, st);
-  if (D == 128) return launch_banded_s<T, 128, NORM>(sh, p, smem, st);
+static rope_status_t launch_banded_d(int D, ShapeId id, const BandedParams &p, size_t smem,
+                                     cudaStream_t st) {
+  if (D == 64) return launch_banded_s<T, 64, NORM>(id, p, smem, st);
+  if (D == 128) return launch_banded_s<T, 128, NORM>(id, p, smem, st);
   if constexpr (sizeof(T) == 2)
-    if (D == 256) return launch_banded_s<T, 256, NORM>(sh, p, smem, st);
+    if (D == 256) return launch_banded_s<T, 256, NORM>(id, p, smem, st);
   return ROPE_ERR_UNSUPPORTED;
 }
 
 static rope_status_t launch_banded(int dtype, int D, bool norm, BandedParams &p,
                                    cudaStream_t st) {
   p.elem_bytes = elem_bytes(dtype);
-  const BandedShape sh = pick_shape(p, norm);
-  const size_t smem = layout_banded(p, D, norm, sh);
+  const ShapeId id = pick_shape(p, D, norm);
+  const size_t smem = layout_banded(p, D, norm, shape_of(id));
   if (smem > 227 * 1024) return ROPE_ERR_UNSUPPORTED;
   if (dtype == ROPE_DTYPE_BF16)
-    return norm ? launch_banded_d<__nv_bfloat16, true>(D, sh, p, smem, st)
-                : launch_banded_d<__nv_bfloat16, false>(D, sh, p, smem, st);
+    return norm ? launch_banded_d<__nv_bfloat16, true>(D, id, p, smem, st)
+                : launch_banded_d<__nv_bfloat16, false>(D, id, p, smem, st);
   if (dtype == ROPE_DTYPE_F16)
-    return norm ? launch_banded_d<__half, true>(D, sh, p, smem, st)
-                : launch_banded_d<__half, false>(D, sh, p, smem, st);
+    return norm ? launch_banded_d<__half, true>(D, id, p, smem, st)
+                : launch_banded_d<__half, false>(D, id, p, smem, st);
   if (dtype == ROPE_DTYPE_F32)
-    return norm ? launch_banded_d<float, true>(D, sh, p, smem, st)
-                : launch_banded_d<float, false>(D, sh, p, smem, st);
+    return norm ? launch_banded_d<float, true>(D, id, p, smem, st)
+                : launch_banded_d<float, false>(D, id, p, smem, st);
   return ROPE_ERR_UNSUPPORTED;
 }
 
@@ -357,17 +375,27 @@ static rope_status_t launch_bshd_d(int D, const BshdParams &p, cudaStream_t st) 
   return ROPE_ERR_UNSUPPORTED;
 }
 
-constexpr int kRaddRing = 96 << 10;  // shared memory of a radd CTA's stage ring
+// Launch shape of the radd kernel (consumer warps, store lag, stage-ring shared memory),
+// measured on B200 over the radd workload: three stages a CTA and four CTAs an SM (65.7 us)
+// beat four stages and three CTAs (76.0 us); the producer and storer threads of more CTAs
+// keep more bulk copies in flight.
+#ifndef ROPE_RADD_CW
+#define ROPE_RADD_CW 4
+#define ROPE_RADD_LAG 0
+#define ROPE_RADD_RING 48
+#endif
+constexpr BandedShape kRaddShape = {ROPE_RADD_CW, ROPE_RADD_LAG, ROPE_RADD_RING};
 
 static size_t layout_radd(RaddParams &p, int D, int eb) {
-  const int kStageTarget = kRaddRing;
+  const int kStageTarget = kRaddShape.ring_kb << 10;
   p.stage_bytes = (int32_t)round_up(4LL * p.n_kv * D * eb, 128);
   int S = (int)(kStageTarget / p.stage_bytes);
-  S = S < 2 ? 2 : (S > kMaxStages ? kMaxStages : S);
+  // the storer holds up to lag + 1 stages; keep at least two for loading / compute
+  S = S < kRaddShape.lag + 3 ? kRaddShape.lag + 3 : (S > kMaxStages ? kMaxStages : S);
   p.S = S;
   int64_t total = (int64_t)S * p.stage_bytes;
   p.bar_off = (int32_t)total;
-  total += 2 * S * 8;
+  total += 3 * S * 8;  // full, done, empty
   p.meta_off = (int32_t)round_up(total, 16);
   total = p.meta_off + S * (int64_t)sizeof(RaddMeta);
   p.offs_off = (int32_t)round_up(total, 16);
@@ -379,12 +407,13 @@ static size_t layout_radd(RaddParams &p, int D, int eb) {
 template <typename T, int D>
 static rope_status_t launch_radd_t(const RaddParams &p, size_t smem, cudaStream_t st) {
   static ShapeCache cache;
-  auto kern = radd_kernel<T, D>;
-  const int occ = resident_ctas(kern, kRaddThreads, smem, cache);
+  constexpr int kThreads = radd_threads<kRaddShape.cw>();
+  auto kern = radd_kernel<T, D, kRaddShape.cw, kRaddShape.lag>;
+  const int occ = resident_ctas(kern, kThreads, smem, cache);
   if (occ <= 0) return ROPE_ERR_UNSUPPORTED;
   const int64_t slots = (int64_t)sm_count() * occ;
   const int grid = (int)(slots < p.T ? slots : p.T);
-  return launch(kern, grid, kRaddThreads, smem, st, p);
+  return launch(kern, grid, kThreads, smem, st, p);
 }
 
 template <typename T>
