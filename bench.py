@@ -175,9 +175,15 @@ def bytes_ragged(w) -> int:
 
 
 def bytes_dual(w) -> int:
+    """Per band: Q heads read and written, K heads read (from the input, or from the cache
+    when updated in place) and written, V heads (when stored) read and written; plus the
+    distinct freqs rows."""
     D, eb = w.main_cache.head_dim, w.input.element_size()
-    heads = (w.main_q_heads + 2 * w.main_cache.n_kv_heads + w.index_q_heads +
-             w.index_cache.n_kv_heads)
+    heads = 0
+    for nq, kv, cols in ((w.main_q_heads, w.main_cache, w.main_cols),
+                         (w.index_q_heads, w.index_cache, w.index_cols)):
+        if kv is not None:
+            heads += nq + kv.n_kv_heads + (kv.n_kv_heads if cols[2] >= 0 else 0)
     return w.total_tokens * 2 * heads * D * eb + freqs_bytes(
         w.rope, positions_ragged(w.lengths, w.main_cache.cache_lengths.tolist()))
 
@@ -202,7 +208,9 @@ def bytes_bshd(w) -> int:
 WORKLOADS = {
     "llama3_8b_prefill": "rope_split_store_paged_ragged",
     "per_head_norm": "fused_qk_rmsnorm_rope_paged",
+    "per_head_norm_multiply_after_cast": "fused_qk_rmsnorm_rope_paged",
     "dual_band_minimax": "fused_dual_qk_rmsnorm_rope_paged",
+    "dual_band_minimax_in_place": "fused_dual_qk_rmsnorm_rope_paged",
     "radd_minimax": "kv_cache_radd",
     "decode_bshd": "qk_rope_bshd_continuous",
 }
@@ -218,7 +226,10 @@ class Case:
 def make_workload(name, seed):
     import workloads as W
     return {"llama3_8b_prefill": W.llama3_8b_prefill, "per_head_norm": W.per_head_norm,
-            "dual_band_minimax": W.dual_band_minimax, "radd_minimax": W.radd_minimax,
+            "per_head_norm_multiply_after_cast": W.per_head_norm,
+            "dual_band_minimax": W.dual_band_minimax,
+            "dual_band_minimax_in_place": W.dual_band_minimax_in_place,
+            "radd_minimax": W.radd_minimax,
             "decode_bshd": W.decode_bshd}[name](seed)
 
 
@@ -260,7 +271,8 @@ def make_case(name, seed, dev, w=None, sched=True):
     def pinned(t):
         return t.contiguous().pin_memory()
 
-    if name in ("llama3_8b_prefill", "per_head_norm"):
+    if name in ("llama3_8b_prefill", "per_head_norm", "per_head_norm_multiply_after_cast"):
+        mbc = 0 if name.endswith("multiply_after_cast") else 1
         w = w or make_workload(name, seed)
         kv = w.cache
         storage = d(kv.storage)
@@ -283,15 +295,15 @@ def make_case(name, seed, dev, w=None, sched=True):
             qg, kg = d(w.q_gamma), d(w.k_gamma)
             args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
                     offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), qg.data_ptr(),
-                    kg.data_ptr(), ctypes.c_float(w.epsilon), ctypes.c_float(w.weight_offset), 1,
-                    w.layer_idx, q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(),
+                    kg.data_ptr(), ctypes.c_float(w.epsilon), ctypes.c_float(w.weight_offset),
+                    mbc, w.layer_idx, q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(),
                     sched_ptr, stream.cuda_stream)
             c.step = bind(lib.fused_qk_rmsnorm_rope_paged, args, c.entry_point)
 
             def call():
                 rs.fused_qk_rmsnorm_rope_paged(qkv, w.n_q_heads, offs, fr, cache, qg, kg,
                                                w.epsilon, w.weight_offset, w.layer_idx, q_out,
-                                               True, c.err, sched=c.sched)
+                                               bool(mbc), c.err, sched=c.sched)
         c.tokens = w.total_tokens
         c.alg_bytes = bytes_ragged(w)
         c.e2e_in = [(pinned(w.qkv), qkv), (pinned(w.offsets), offs),
@@ -305,9 +317,10 @@ def make_case(name, seed, dev, w=None, sched=True):
                     "batch": len(w.lengths), "lengths": w.lengths,
                     "rope": f"{'interleaved' if w.rope.interleaved else 'half-split'}, "
                             f"rope_dim {w.rope.rope_dim}, freqs_cis {w.rope.dtype}",
-                    "rmsnorm": w.q_gamma is not None}
+                    "rmsnorm": w.q_gamma is not None,
+                    "multiply_before_cast": bool(mbc)}
         c.workload = w
-    elif name == "dual_band_minimax":
+    elif name in ("dual_band_minimax", "dual_band_minimax_in_place"):
         w = w or make_workload(name, seed)
         inp, offs = d(w.input), d(w.offsets)
         ms, ist = d(w.main_cache.storage), d(w.index_cache.storage)
@@ -344,7 +357,7 @@ def make_case(name, seed, dev, w=None, sched=True):
                     "index_heads": [w.index_q_heads, w.index_cache.n_kv_heads],
                     "head_dim": w.main_cache.head_dim, "rope_dim": w.rope.rope_dim,
                     "page_size": [w.main_cache.page_size, w.index_cache.page_size],
-                    "batch": len(w.lengths)}
+                    "batch": len(w.lengths), "k_in_place": w.main_cols[1] < 0}
         c.workload = w
     elif name == "radd_minimax":
         w = w or make_workload(name, seed)
@@ -607,7 +620,11 @@ def run_ours(args):
 
 KERNELS = {"llama3_8b_prefill": "banded_store_kernel<bf16, head_dim 128, no norm>",
            "per_head_norm": "banded_store_kernel<bf16, head_dim 128, rmsnorm>",
+           "per_head_norm_multiply_after_cast":
+               "banded_store_kernel<bf16, head_dim 128, rmsnorm, multiply after cast>",
            "dual_band_minimax": "banded_store_kernel<bf16, head_dim 128, rmsnorm> (two bands)",
+           "dual_band_minimax_in_place":
+               "banded_store_kernel<bf16, head_dim 128, rmsnorm> (two bands, K in place)",
            "radd_minimax": "radd_kernel<bf16, head_dim 128>",
            "decode_bshd": "bshd_rope_kernel<bf16, head_dim 128>"}
 

@@ -160,9 +160,12 @@ typedef struct {
 } rope_cont_cache_t;
 
 /* One band of the dual per-head RMSNorm + RoPE launch: its Q heads start at column q_col,
- * its K heads at k_col and its V heads at v_col (v_col < 0: the band's cache is K-only) of
- * the token-major `input` (the pages' per-band Q read lambdas become a base pointer, a row
- * stride and column offsets).  q_gamma / k_gamma: [head_dim] in the element type, shared by
+ * its K heads at k_col and its V heads at v_col (v_col < 0: the band's cache is K-only, or
+ * its V is not stored) of the token-major `input` (the pages' per-band Q read lambdas become
+ * a base pointer, a row stride and column offsets).  k_col < 0: the band's K heads are not
+ * in the input; they are read from the token's cache slot, normalised, rotated and written
+ * back to that slot (the key cache updated in place, fused_dual_qk_rms_norm_rope_ragged_paged
+ * first paragraph).  q_gamma / k_gamma: [head_dim] in the element type, shared by
  * all Q (K) heads of the band.  epsilon: the band's RMSNorm epsilon.  q_out: [T, n_q_heads *
  * head_dim] rows with stride q_out_row_stride. */
 typedef struct {
@@ -203,8 +206,11 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
  * becomes x * rsqrt(mean(x^2) + epsilon) * (gamma + weight_offset) with gamma = q_gamma
  * (k_gamma); RoPE then rotates that normalised row (no rounding in between).
  * weight_offset is a scalar of the element type (the page's Scalar[dtype]): it is rounded
- * to the element type first.  multiply_before_cast must be 1 (the normalised row is
- * multiplied by gamma before any rounding); 0 returns ROPE_ERR_UNSUPPORTED. */
+ * to the element type first.  multiply_before_cast != 0: the normalised row is multiplied
+ * by gamma before any rounding.  multiply_before_cast == 0: the normalised value
+ * x * rsqrt(mean(x^2) + epsilon) is rounded to the element type first and then multiplied
+ * by (gamma + weight_offset); RoPE follows in float32 and the result is rounded once more
+ * (the pages name the flag but do not define it; this is the reading taken). */
 rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_stride,
                                           int32_t total_tokens, int32_t n_q_heads,
                                           const uint32_t *input_row_offsets, int32_t batch,
@@ -224,7 +230,8 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
  * rope geometry must agree across bands: same element type and head_dim in both caches
  * (else ROPE_ERR_INVALID_ARG, the runtime form of the page's compile-time assert).  The
  * result equals fused_qk_rmsnorm_rope_paged on the main band followed by the same on the
- * index band. */
+ * index band.  index_band may be NULL: the launch then has the main band alone (the general
+ * single-band form, e.g. for K updated in place). */
 rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band,
                                                const rope_norm_band_t *index_band,
                                                const uint32_t *input_row_offsets,

@@ -11,9 +11,14 @@ returns the data-dependent error bits (``ERR_*``) it met; 0 means every token wa
 
 Parity status of the functions (what pins each one is stated in the test-suite):
   rope_split_store_paged_ragged, fused_qk_rmsnorm_rope_paged (multiply_before_cast=1),
-  fused_dual_qk_rmsnorm_rope_paged, qk_rope_bshd_continuous, kv_cache_radd: pinned.
-  multiply_before_cast=0 and the choice of rotated columns under partial RoPE are
-  readings of open points; they are pinned only against the reading they implement.
+  fused_dual_qk_rmsnorm_rope_paged, qk_rope_bshd_continuous, kv_cache_radd, and bands whose
+  K is updated in place (k_col < 0; pinned against the store mode on a cache that holds the
+  input's K): pinned.
+  multiply_before_cast=0: parity unpinned (the pages name the flag without defining it; the
+  reading implemented rounds the normalised value to the element type before the gamma
+  multiply, and only its reduction to the plain op at unit gamma is checked).
+  The choice of rotated columns under partial RoPE is a reading of an open point; it is
+  pinned only against the reading it implements.
 """
 from __future__ import annotations
 
@@ -166,7 +171,8 @@ class Band:
     input: np.ndarray           # 2-D [tokens, columns]
     q_col: int
     k_col: int
-    v_col: int                  # -1: K-only cache
+    v_col: int                  # -1: K-only cache (or V not stored)
+    # k_col -1: K heads read from the token's cache slot and updated there (in place)
     n_q_heads: int
     cache: PagedCache
     q_gamma: np.ndarray

@@ -203,7 +203,9 @@ static void rmsnorm_head(int32_t dtype, double *y, int32_t D, const void *gamma,
 /* ------------------------------------------------------------------ banded store op -- */
 
 /* One band: for every token row, optionally RMSNorm then RoPE its Q heads into q_out,
- * its K heads into the band's cache, and copy its V heads into the cache. */
+ * its K heads into the band's cache, and copy its V heads into the cache.  With k_col < 0
+ * the K heads are not in the input: they are read from the token's cache slot and updated
+ * there in place ([P4]: the key caches are updated in place). */
 static uint32_t apply_band(int32_t dtype, orc_band *bd, const uint32_t *offs, int32_t batch,
                            int32_t T, const orc_rope *rope, int32_t do_norm,
                            double weight_offset, int32_t mbc, uint32_t layer) {
@@ -235,8 +237,11 @@ static uint32_t apply_band(int32_t dtype, orc_band *bd, const uint32_t *offs, in
       rope_head(y, D, rope, cs);
       for (int32_t d = 0; d < D; ++d) orc_encode(dtype, bd->q_out, row * bd->q_out_row_stride + (int64_t)h * D + d, y[d]);
     }
-    for (int32_t h = 0; h < Hk; ++h) { /* K heads -> K cache */
-      for (int32_t d = 0; d < D; ++d) y[d] = orc_decode(dtype, bd->input, in_row + bd->k_col + (int64_t)h * D + d);
+    for (int32_t h = 0; h < Hk; ++h) { /* K heads -> K cache (k_col < 0: K is the cache's) */
+      for (int32_t d = 0; d < D; ++d)
+        y[d] = bd->k_col >= 0
+                   ? orc_decode(dtype, bd->input, in_row + bd->k_col + (int64_t)h * D + d)
+                   : orc_decode(c->dtype, c->k, base + h * c->head_stride + d);
       if (do_norm) rmsnorm_head(dtype, y, D, bd->k_gamma, eps, weight_offset, mbc);
       rope_head(y, D, rope, cs);
       for (int32_t d = 0; d < D; ++d) orc_encode(c->dtype, c->k, base + h * c->head_stride + d, y[d]);

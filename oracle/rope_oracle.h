@@ -16,6 +16,10 @@
  * Arithmetic: every value is widened to double, every step is evaluated in double in the
  * order the definition states, and each output element is rounded exactly once, with
  * round-to-nearest-even, to the output element type.
+ *
+ * multiply_before_cast = 0 is parity unpinned: the pages name the flag without defining it.
+ * The reading implemented rounds the normalised value to the element type before the gamma
+ * multiply (a second rounding ahead of the final one).
  */
 #ifndef ROPE_ORACLE_H
 #define ROPE_ORACLE_H
@@ -77,7 +81,8 @@ typedef struct {
 typedef struct {
   const void *input;       /* token-major rows */
   int64_t input_row_stride;
-  int64_t q_col, k_col, v_col; /* first column of Q / K / V heads; v_col < 0: K-only */
+  int64_t q_col, k_col, v_col; /* first column of Q / K / V heads; v_col < 0: K-only;
+                                  k_col < 0: K is read from the cache slot (in place) */
   int32_t n_q_heads;
   orc_paged_cache *cache;
   const void *q_gamma, *k_gamma; /* [head_dim] each, element type = dtype */

@@ -72,20 +72,29 @@ def oracle_ragged_store(w: "W.RaggedStore", dtype: str = "bf16",
     return OracleResult(q_out=q_out, storage=store, written=written, err=err)
 
 
-def oracle_dual(w: "W.DualBand", dtype: str = "bf16") -> OracleResult:
+def oracle_dual(w: "W.DualBand", dtype: str = "bf16",
+                multiply_before_cast: bool = True) -> OracleResult:
+    """The two-band op, or the single-band op when the workload has no index band."""
     inp = bits(w.input)
-    ms, ist = bits(w.main_cache.storage), bits(w.index_cache.storage)
-    qm, qi = bits(w.q_main_out), bits(w.q_index_out)
+    ms = bits(w.main_cache.storage)
+    qm = bits(w.q_main_out)
     wm = np.zeros(w.main_cache.num_pages * w.main_cache.page_size, dtype=np.uint8)
-    wi = np.zeros(w.index_cache.num_pages * w.index_cache.page_size, dtype=np.uint8)
-    g = [bits(x) for x in w.gammas]
+    g = [None if x is None else bits(x) for x in w.gammas]
     main = oracle.Band(inp, *w.main_cols, w.main_q_heads, oracle_paged(w.main_cache, ms), g[0],
                        g[1], w.main_eps, qm, wm)
+    if w.index_cache is None:
+        err = oracle.fused_qk_rmsnorm_rope_paged(main, bits(w.offsets), oracle_rope(w.rope),
+                                                 w.weight_offset, multiply_before_cast,
+                                                 w.layer_idx, dtype)
+        return OracleResult(q_main_out=qm, main_storage=ms, main_written=wm, err=err)
+    ist = bits(w.index_cache.storage)
+    qi = bits(w.q_index_out)
+    wi = np.zeros(w.index_cache.num_pages * w.index_cache.page_size, dtype=np.uint8)
     index = oracle.Band(inp, *w.index_cols, w.index_q_heads, oracle_paged(w.index_cache, ist),
                         g[2], g[3], w.index_eps, qi, wi)
     err = oracle.fused_dual_qk_rmsnorm_rope_paged(main, index, bits(w.offsets),
-                                                  oracle_rope(w.rope), w.weight_offset, True,
-                                                  w.layer_idx, dtype)
+                                                  oracle_rope(w.rope), w.weight_offset,
+                                                  multiply_before_cast, w.layer_idx, dtype)
     return OracleResult(q_main_out=qm, q_index_out=qi, main_storage=ms, index_storage=ist,
                         main_written=wm, index_written=wi, err=err)
 

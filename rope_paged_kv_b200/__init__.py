@@ -312,15 +312,16 @@ def fused_qk_rmsnorm_rope_paged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
         "fused_qk_rmsnorm_rope_paged")
 
 
-def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: NormBand,
+def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: Optional[NormBand],
                                      input_row_offsets, total_tokens, freqs: Freqs,
                                      weight_offset, layer_idx, multiply_before_cast=True,
                                      err_word=None, stream=None, sched=None) -> None:
     offs = _idx(input_row_offsets)
     keep: list = []
-    m, i, f = main_band.c(keep), index_band.c(keep), freqs.c()
+    m, f = main_band.c(keep), freqs.c()
+    i = None if index_band is None else ctypes.byref(index_band.c(keep))
     _check(_lib.fused_dual_qk_rmsnorm_rope_paged(
-        ctypes.byref(m), ctypes.byref(i), offs.data_ptr(), offs.shape[0] - 1, total_tokens,
+        ctypes.byref(m), i, offs.data_ptr(), offs.shape[0] - 1, total_tokens,
         ctypes.byref(f), weight_offset, int(bool(multiply_before_cast)), layer_idx,
         _ptr(err_word), _sched(sched), _stream(stream)), "fused_dual_qk_rmsnorm_rope_paged")
 

@@ -51,6 +51,7 @@ struct BandDev {
   int64_t seg_col[3];
   int32_t seg_bytes[3], seg_dst[3];
   int32_t kv_contig;  // a slot's heads are adjacent in the cache (one store per plane)
+  int32_t k_inplace;  // K heads come from the token's cache slot, not from the input
 };
 
 struct BandedParams {
@@ -65,6 +66,7 @@ struct BandedParams {
   uint32_t layer;
   uint32_t *err;
   float weight_offset;
+  int32_t mbc;  // multiply_before_cast: 0 rounds the normalised value before the gamma multiply
   // dynamic shared memory layout
   int32_t S, stage_bytes, f_row_bytes, staged, elem_bytes;
   int32_t bar_off, meta_off, gamma_off, offs_off, items_off;
@@ -346,6 +348,17 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
               for (int q = 0; q < bd.nseg; ++q)
                 bulk_g2s(st + bd.seg_dst[q], row + bd.seg_col[q] * EB, (uint32_t)bd.seg_bytes[q],
                          &full[s]);
+              if (bd.k_inplace && bd.n_kv > 0) {  // K from the slot it is updated in
+                const unsigned char *kc =
+                    reinterpret_cast<const unsigned char *>(bd.cache.k) + mj.kv_base[k] * EB;
+                unsigned char *kd = st + bd.smem_off + bd.n_q * D * EB;
+                if (bd.kv_contig)
+                  bulk_g2s(kd, kc, (uint32_t)(bd.n_kv * D * EB), &full[s]);
+                else
+                  for (int h = 0; h < bd.n_kv; ++h)
+                    bulk_g2s(kd + h * D * EB, kc + (int64_t)h * bd.cache.head_stride * EB,
+                             (uint32_t)(D * EB), &full[s]);
+              }
               if (p.f_row_bytes)
                 bulk_g2s(st + bd.f_off,
                          reinterpret_cast<const unsigned char *>(p.rope.table) +
@@ -589,14 +602,29 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
           for (int msk = L / 2; msk > 0; msk >>= 1) ss += __shfl_xor_sync(gmask, ss, msk);
           const float r = rsqrtf(ss * (1.0f / D) + bd.eps);
           const float2 rr = make_float2(r, r);
+          if (p.mbc) {
 #pragma unroll
-          for (int e = 0; e < N; e += 2) {
-            const float2 ya = __fmul2_rn(make_float2(xa[e], xa[e + 1]),
-                                         __fmul2_rn(rr, make_float2(ga[e], ga[e + 1])));
-            const float2 yb = __fmul2_rn(make_float2(xb[e], xb[e + 1]),
-                                         __fmul2_rn(rr, make_float2(gb[e], gb[e + 1])));
-            xa[e] = ya.x; xa[e + 1] = ya.y;
-            xb[e] = yb.x; xb[e + 1] = yb.y;
+            for (int e = 0; e < N; e += 2) {
+              const float2 ya = __fmul2_rn(make_float2(xa[e], xa[e + 1]),
+                                           __fmul2_rn(rr, make_float2(ga[e], ga[e + 1])));
+              const float2 yb = __fmul2_rn(make_float2(xb[e], xb[e + 1]),
+                                           __fmul2_rn(rr, make_float2(gb[e], gb[e + 1])));
+              xa[e] = ya.x; xa[e + 1] = ya.y;
+              xb[e] = yb.x; xb[e + 1] = yb.y;
+            }
+          } else {  // the normalised value is rounded to the element type, then scaled
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+              xa[e] *= r;
+              xb[e] *= r;
+            }
+            VT::widen(VT::narrow(xa), xa);
+            VT::widen(VT::narrow(xb), xb);
+#pragma unroll
+            for (int e = 0; e < N; ++e) {
+              xa[e] *= ga[e];
+              xb[e] *= gb[e];
+            }
           }
         }
         if (inter) {

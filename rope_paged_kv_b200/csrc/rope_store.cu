@@ -200,27 +200,28 @@ static float round_to_elem(float x, int dtype) {
 }
 
 // Validate one band and fill its device descriptor (staging segments included; the
-// band's stage offset is set by the caller).
+// band's stage offset is set by the caller).  k_col < 0: K is read from the cache slot.
 static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride, int64_t q_col,
                                int64_t k_col, int64_t v_col, int32_t n_q,
                                const rope_paged_cache_t *kv, const void *qg, const void *kg,
                                float eps, void *q_out, int64_t q_out_stride, int dtype,
                                uint32_t layer, bool norm) {
   if (input == nullptr || q_out == nullptr || n_q < 0 || in_stride < 0 || q_out_stride < 0 ||
-      q_col < 0 || k_col < 0)
+      q_col < 0)
     return ROPE_ERR_INVALID_ARG;
+  const bool k_inplace = k_col < 0;
   if (norm && (qg == nullptr || kg == nullptr)) return ROPE_ERR_INVALID_ARG;
   rope_status_t s = check_paged(kv, dtype, layer, v_col >= 0, &bd->cache);
   if (s != ROPE_OK) return s;
   const int64_t D = kv->head_dim, Hk = kv->n_kv_heads;
   const int eb = elem_bytes(dtype);
   const int64_t nv = v_col >= 0 ? Hk : 0;
-  if (in_stride < q_col + n_q * D || in_stride < k_col + Hk * D ||
+  if (in_stride < q_col + n_q * D || (!k_inplace && in_stride < k_col + Hk * D) ||
       (v_col >= 0 && in_stride < v_col + Hk * D) || q_out_stride < n_q * D)
     return ROPE_ERR_INVALID_ARG;
   if (!aligned16(input) || !aligned16(q_out) || !stride16(in_stride, eb) ||
-      !stride16(q_out_stride, eb) || !stride16(q_col, eb) || !stride16(k_col, eb) ||
-      (v_col >= 0 && !stride16(v_col, eb)))
+      !stride16(q_out_stride, eb) || !stride16(q_col, eb) ||
+      (!k_inplace && !stride16(k_col, eb)) || (v_col >= 0 && !stride16(v_col, eb)))
     return ROPE_ERR_UNSUPPORTED;
   bd->input = input;
   bd->in_stride = in_stride;
@@ -236,13 +237,20 @@ static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride
   bd->k_gamma = kg;
   bd->eps = eps;
   bd->kv_contig = kv->head_stride == D ? 1 : 0;
-  // staging segments: Q, K, V blocks (merged when adjacent in the input row)
+  bd->k_inplace = k_inplace ? 1 : 0;
+  // staging segments: Q, K, V blocks (merged when adjacent in the input row); an in-place
+  // K block keeps its place in the stage but is loaded from the cache
   const int64_t cols[3] = {q_col, k_col, v_col};
   const int64_t cnt[3] = {n_q * D, Hk * D, nv * D};
   int nseg = 0;
   int64_t dst = 0, next_col = -1;
   for (int q = 0; q < 3; ++q) {
     if (cnt[q] == 0) continue;
+    if (q == 1 && k_inplace) {
+      dst += cnt[q] * eb;
+      next_col = -1;
+      continue;
+    }
     if (nseg > 0 && cols[q] == next_col) {
       bd->seg_bytes[nseg - 1] += (int32_t)(cnt[q] * eb);
     } else {
@@ -518,8 +526,8 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
   if (batch > kv->n_seqs || n_q_heads < 0) return ROPE_ERR_INVALID_ARG;
-  if (multiply_before_cast != 1) return ROPE_ERR_UNSUPPORTED;
   BandedParams p{};
+  p.mbc = multiply_before_cast != 0;
   s = check_freqs(freqs, dtype, D, &p.rope);
   if (s != ROPE_OK) return s;
   const int64_t Hq = n_q_heads, Hk = kv->n_kv_heads;
@@ -549,23 +557,26 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
                                                uint32_t *err_word, uint32_t *sched,
                                                rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
-  if (main_band == nullptr || index_band == nullptr || main_band->cache == nullptr ||
-      index_band->cache == nullptr || !sched_ok(sched))
+  // index_band == NULL: a launch of the main band alone
+  const int n_bands = index_band == nullptr ? 1 : 2;
+  if (main_band == nullptr || main_band->cache == nullptr ||
+      (index_band != nullptr && index_band->cache == nullptr) || !sched_ok(sched))
     return ROPE_ERR_INVALID_ARG;
-  const rope_paged_cache_t *mc = main_band->cache, *ic = index_band->cache;
+  const rope_paged_cache_t *mc = main_band->cache;
+  const rope_paged_cache_t *ic = n_bands == 2 ? index_band->cache : mc;
   // the rope geometry must agree across the bands
   if (mc->dtype != ic->dtype || mc->head_dim != ic->head_dim) return ROPE_ERR_INVALID_ARG;
   const int dtype = mc->dtype, D = mc->head_dim;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
   if (batch > mc->n_seqs || batch > ic->n_seqs) return ROPE_ERR_INVALID_ARG;
-  if (multiply_before_cast != 1) return ROPE_ERR_UNSUPPORTED;
   BandedParams p{};
+  p.mbc = multiply_before_cast != 0;
   s = check_freqs(freqs, dtype, D, &p.rope);
   if (s != ROPE_OK) return s;
   const rope_norm_band_t *bands[2] = {main_band, index_band};
-  int32_t rows[2];
-  for (int k = 0; k < 2; ++k) {
+  int32_t rows[2] = {0, 0};
+  for (int k = 0; k < n_bands; ++k) {
     const rope_norm_band_t *b = bands[k];
     s = fill_band(&p.band[k], b->input, b->input_row_stride, b->q_col, b->k_col, b->v_col,
                   b->n_q_heads, b->cache, b->q_gamma, b->k_gamma, b->epsilon, b->q_out,
@@ -573,7 +584,7 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
     if (s != ROPE_OK) return s;
     rows[k] = p.band[k].n_q + p.band[k].n_kv;
   }
-  p.n_bands = 2;
+  p.n_bands = n_bands;
   p.work0 = rows[0];
   p.work_total = rows[0] + rows[1];
   p.offs = input_row_offsets;

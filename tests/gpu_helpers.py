@@ -77,51 +77,57 @@ def stage_ragged(w: W.RaggedStore) -> Staged:
     return s
 
 
-def launch_ragged(w: W.RaggedStore, s: Staged, stream=None) -> None:
+def launch_ragged(w: W.RaggedStore, s: Staged, stream=None, multiply_before_cast=True) -> None:
     if w.q_gamma is None:
         rs.rope_split_store_paged_ragged(s.qkv, w.n_q_heads, s.offs, s.freqs, s.kv,
                                          w.layer_idx, s.q_out, s.err, stream, sched_of(s))
     else:
         rs.fused_qk_rmsnorm_rope_paged(s.qkv, w.n_q_heads, s.offs, s.freqs, s.kv, s.q_gamma,
                                        s.k_gamma, w.epsilon, w.weight_offset, w.layer_idx,
-                                       s.q_out, True, s.err, stream, sched_of(s))
+                                       s.q_out, multiply_before_cast, s.err, stream,
+                                       sched_of(s))
 
 
-def run_ragged(w: W.RaggedStore):
+def run_ragged(w: W.RaggedStore, multiply_before_cast=True):
     s = stage_ragged(w)
-    launch_ragged(w, s)
+    launch_ragged(w, s, multiply_before_cast=multiply_before_cast)
     torch.cuda.synchronize()
     return s
 
 
 def stage_dual(w: W.DualBand) -> Staged:
+    """The dual-band workload staged; a workload without an index band stages the main
+    band alone (s.index is None)."""
     s = Staged()
     s.input = to_dev(w.input)
     s.offs = to_dev(w.offsets)
     s.main_storage = to_dev(w.main_cache.storage)
-    s.index_storage = to_dev(w.index_cache.storage)
-    s.q_main_out, s.q_index_out = to_dev(w.q_main_out), to_dev(w.q_index_out)
-    g = [to_dev(x) for x in w.gammas]
+    s.q_main_out = to_dev(w.q_main_out)
+    g = [None if x is None else to_dev(x) for x in w.gammas]
     s.main = rs.NormBand(s.input, *w.main_cols, w.main_q_heads,
                          paged(w.main_cache, s.main_storage), g[0], g[1], w.main_eps,
                          s.q_main_out)
-    s.index = rs.NormBand(s.input, *w.index_cols, w.index_q_heads,
-                          paged(w.index_cache, s.index_storage), g[2], g[3], w.index_eps,
-                          s.q_index_out)
+    s.index = None
+    if w.index_cache is not None:
+        s.index_storage = to_dev(w.index_cache.storage)
+        s.q_index_out = to_dev(w.q_index_out)
+        s.index = rs.NormBand(s.input, *w.index_cols, w.index_q_heads,
+                              paged(w.index_cache, s.index_storage), g[2], g[3], w.index_eps,
+                              s.q_index_out)
     s.freqs = freqs(w.rope)
     s.err = err_word()
     return s
 
 
-def launch_dual(w: W.DualBand, s: Staged, stream=None) -> None:
+def launch_dual(w: W.DualBand, s: Staged, stream=None, multiply_before_cast=True) -> None:
     rs.fused_dual_qk_rmsnorm_rope_paged(s.main, s.index, s.offs, w.total_tokens, s.freqs,
-                                        w.weight_offset, w.layer_idx, True, s.err, stream,
-                                        sched_of(s))
+                                        w.weight_offset, w.layer_idx, multiply_before_cast,
+                                        s.err, stream, sched_of(s))
 
 
-def run_dual(w: W.DualBand):
+def run_dual(w: W.DualBand, multiply_before_cast=True):
     s = stage_dual(w)
-    launch_dual(w, s)
+    launch_dual(w, s, multiply_before_cast=multiply_before_cast)
     torch.cuda.synchronize()
     return s
 

@@ -37,19 +37,26 @@ def bf16_ulp(v: np.ndarray) -> np.ndarray:
     return np.exp2(e - 7)
 
 
-def assert_close_bf16(got_bits: np.ndarray, want_bits: np.ndarray, what: str,
-                      abs_tol: float = 1e-3, dtype: str = "bf16"):
-    """|got - want| <= max(1 ulp of want, abs_tol) elementwise (want = oracle, already
-    rounded once); returns the fraction of bit-identical elements."""
-    g, w = values(got_bits, dtype), values(want_bits, dtype)
+def ulp_of(v: np.ndarray, dtype: str) -> np.ndarray:
+    """Spacing of the element type's numbers at |v|."""
     if dtype == "bf16":
-        ulp = bf16_ulp(w)
-    elif dtype == "f16":
-        a = np.maximum(np.abs(w), 2.0 ** -14)
-        ulp = np.exp2(np.floor(np.log2(a)) - 10)
-    else:
-        ulp = np.spacing(np.abs(w).astype(np.float32)).astype(np.float64)
+        return bf16_ulp(v)
+    if dtype == "f16":
+        a = np.maximum(np.abs(v), 2.0 ** -14)
+        return np.exp2(np.floor(np.log2(a)) - 10)
+    return np.spacing(np.abs(v).astype(np.float32)).astype(np.float64)
+
+
+def assert_close_bf16(got_bits: np.ndarray, want_bits: np.ndarray, what: str,
+                      abs_tol: float = 1e-3, dtype: str = "bf16", extra=None):
+    """|got - want| <= max(1 ulp of want, abs_tol) (+ extra, elementwise, where a reading
+    adds an intermediate rounding) elementwise (want = oracle, already rounded once);
+    returns the fraction of bit-identical elements."""
+    g, w = values(got_bits, dtype), values(want_bits, dtype)
+    ulp = ulp_of(w, dtype)
     tol = np.maximum(ulp, abs_tol)
+    if extra is not None:
+        tol = tol + extra
     same = _as_bits(np.ascontiguousarray(got_bits)) == _as_bits(np.ascontiguousarray(want_bits))
     bad = ~(same | (np.abs(g - w) <= tol))
     if bad.any():
@@ -83,7 +90,7 @@ def paged_rows_mask(kv: W.PagedKV, written: np.ndarray, layer_idx: int) -> np.nd
 
 def compare_paged_cache(kv: W.PagedKV, got_storage: np.ndarray, want_storage: np.ndarray,
                         written: np.ndarray, layer_idx: int, fp_cols_k: np.ndarray,
-                        what: str, v_exact: bool = True):
+                        what: str, v_exact: bool = True, k_extra=None):
     """Rows the oracle did not write: bit-identical (untouched).  Written K rows: columns in
     fp_cols_k within tolerance, other columns bit-identical.  Written V rows: bit-identical
     (or within tolerance when v_exact is False, for radd the tolerance is still exact)."""
@@ -98,8 +105,9 @@ def compare_paged_cache(kv: W.PagedKV, got_storage: np.ndarray, want_storage: np
     gk, wk = g[kr], w[kr]            # [n, Hk, D]
     exact_cols = ~fp_cols_k
     assert_bits_equal(gk[..., exact_cols], wk[..., exact_cols], f"{what}: K pass-through cols")
+    ek = None if k_extra is None else k_extra.reshape(shp)[kr][..., fp_cols_k]
     frac = assert_close_bf16(gk[..., fp_cols_k], wk[..., fp_cols_k], f"{what}: K roped cols",
-                             dtype=kv.dtype)
+                             dtype=kv.dtype, extra=ek)
     if kv.planes == 2:
         vr = rows.copy()
         vr[:, 0] = False
@@ -179,3 +187,45 @@ def tile_golden(case: dict, head_dim: int = 64) -> dict:
         assert o0 == 0
         c["gamma"] = tile_row(case["gamma"])
     return c
+
+
+# ------------------------------------------- the multiply-after-cast reading's tolerance --
+
+def rope_pairs(head_dim: int, rope: W.RopeSpec) -> np.ndarray:
+    """partner[d] = the column rotated together with column d (d itself if unrotated)."""
+    R = rope.rope_dim
+    o = head_dim - R if rope.rope_col_offset < 0 else rope.rope_col_offset
+    partner = np.arange(head_dim)
+    for i in range(R // 2):
+        a, b = (o + 2 * i, o + 2 * i + 1) if rope.interleaved else (o + i, o + i + R // 2)
+        partner[a], partner[b] = b, a
+    return partner
+
+
+def multiply_after_cast_slack(x: np.ndarray, gamma: np.ndarray, weight_offset: float,
+                              eps: float, dtype: str, rope: W.RopeSpec) -> np.ndarray:
+    """Extra tolerance of multiply_before_cast = 0, elementwise for head rows x [..., D]
+    (float64 values) of the input.  That reading rounds the normalised value n = x * r to the
+    element type before the gamma multiply: both sides round n, the kernel from a float32 n
+    (rsqrtf, float32 products), the oracle from the exact one, so where n lies within a few
+    float32 ulps of a rounding midpoint they may keep neighbouring values of the element
+    type.  Such a flip moves the gamma-scaled value by ulp(n) * |gamma + weight_offset|, and
+    the rotation mixes it into both columns of the pair (|cos|, |sin| <= 1)."""
+    D = x.shape[-1]
+    r = 1.0 / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    n = x * r
+    u = ulp_of(n * (1.0 + 2.0 ** -7), dtype) * np.abs(gamma + weight_offset)
+    partner = rope_pairs(D, rope)
+    rotated = partner != np.arange(D)
+    return np.where(rotated, u + u[..., partner], u)
+
+
+def scatter_slots(kv: W.PagedKV, per_token: np.ndarray, cache_lengths, lengths,
+                  layer_idx: int) -> np.ndarray:
+    """Per-token K-row values [T, Hk, D] placed at the cache rows the tokens map to (K plane
+    of layer_idx), zeros elsewhere: storage-shaped."""
+    out = np.zeros((kv.num_pages, kv.planes, kv.num_layers, kv.page_size, kv.n_kv_heads,
+                    kv.head_dim))
+    for i, (page, slot) in enumerate(W.token_slots(kv, list(cache_lengths), list(lengths))):
+        out[page, 0, layer_idx, slot] = per_token[i]
+    return out

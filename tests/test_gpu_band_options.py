@@ -1,0 +1,64 @@
+"""Band options beyond the store of the named workloads, CUDA path vs the oracle.
+
+K updated in place (a band whose K heads are read from the token's cache slot and written
+back there, V untouched), the single-band launch (no index band), and
+multiply_before_cast = 0 (the normalised value rounded to the element type before the
+gamma multiply).  Tolerances as in test_gpu_parity.py.
+"""
+import pytest
+import torch
+
+import workloads as W
+from test_gpu_parity import _check_dual, check_ragged
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def G():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import gpu_helpers
+    return gpu_helpers
+
+
+def band_case(seed, **kw):
+    base = dict(lengths=[300, 1, 57, 640], cache_lengths=[0, 9, 200, 33], main_q_heads=8,
+                main_kv_heads=2, index_q_heads=2, index_kv_heads=1, head_dim=128,
+                main_page_size=64, index_page_size=32, rope_dim=64, theta=1e4,
+                interleaved=True, max_seq_len=1024)
+    base.update(kw)
+    return W.dual_band(seed, **base)
+
+
+@pytest.mark.parametrize("single", [False, True])
+@pytest.mark.parametrize("interleaved", [True, False])
+def test_k_in_place(G, single, interleaved):
+    w = band_case(41, k_in_place=True, single=single, interleaved=interleaved)
+    _check_dual(G, w, G.run_dual(w))
+
+
+def test_single_band_store(G):
+    w = band_case(42, single=True)
+    _check_dual(G, w, G.run_dual(w))
+
+
+def test_k_in_place_full_size(G):
+    # the dual-band workload with both key caches updated in place (the literal reading)
+    w = W.dual_band_minimax_in_place()
+    _check_dual(G, w, G.run_dual(w))
+
+
+@pytest.mark.parametrize("head_dim,dtype", [(128, "bf16"), (64, "f16"), (128, "f32")])
+def test_multiply_after_cast_ragged(G, head_dim, dtype):
+    w = W.ragged_store(43, lengths=[129, 3, 700], cache_lengths=[0, 17, 64], n_q_heads=8,
+                       n_kv_heads=2, head_dim=head_dim, page_size=32, rope_dim=head_dim // 2,
+                       theta=1e4, interleaved=False, max_seq_len=1024, x_std=2.0, norm=True,
+                       weight_offset=1.0, dtype=dtype)
+    s = G.run_ragged(w, multiply_before_cast=False)
+    check_ragged(G, w, s, multiply_before_cast=False)
+
+
+def test_multiply_after_cast_dual_in_place(G):
+    w = band_case(44, k_in_place=True, x_std=2.0)
+    _check_dual(G, w, G.run_dual(w, multiply_before_cast=False), multiply_before_cast=False)

@@ -28,18 +28,40 @@ def G():
     return gpu_helpers
 
 
-def check_ragged(G, w, s, exact_norm_cols=False):
-    r = H.oracle_ragged_store(w, w.cache.dtype)
+def _head_rows(x, col, heads, D):
+    return x[:, col:col + heads * D].reshape(x.shape[0], heads, D)
+
+
+def _slot_rows(kv, storage_bits, cache_lengths, lengths, layer_idx):
+    """The K rows a band updated in place held before the call, in token order."""
+    v = H.values(storage_bits, kv.dtype).reshape(kv.num_pages, kv.planes, kv.num_layers,
+                                                 kv.page_size, kv.n_kv_heads, kv.head_dim)
+    return np.stack([v[p, 0, layer_idx, sl] for p, sl in
+                     W.token_slots(kv, list(cache_lengths), list(lengths))])
+
+
+def check_ragged(G, w, s, exact_norm_cols=False, multiply_before_cast=True):
+    r = H.oracle_ragged_store(w, w.cache.dtype, multiply_before_cast)
     assert int(s.err.item()) == r.err
-    D, T, Hq = w.cache.head_dim, w.total_tokens, w.n_q_heads
+    D, T, Hq, Hk = w.cache.head_dim, w.total_tokens, w.n_q_heads, w.cache.n_kv_heads
     norm = w.q_gamma is not None
     fpc = np.ones(D, bool) if norm else H.rope_cols(D, w.rope.rope_dim, w.rope.rope_col_offset)
+    eq = ek = None
+    if not multiply_before_cast:  # the reading's intermediate rounding (helpers.py)
+        dt = w.cache.dtype
+        x = H.values(H.bits(w.qkv), dt).reshape(T, -1)
+        gq, gk = H.values(H.bits(w.q_gamma), dt), H.values(H.bits(w.k_gamma), dt)
+        eq = H.multiply_after_cast_slack(_head_rows(x, 0, Hq, D), gq, w.weight_offset,
+                                         w.epsilon, dt, w.rope)[..., fpc]
+        ek = H.scatter_slots(w.cache, H.multiply_after_cast_slack(
+            _head_rows(x, Hq * D, Hk, D), gk, w.weight_offset, w.epsilon, dt, w.rope),
+            w.cache.cache_lengths.tolist(), w.lengths, w.layer_idx)
     q = H.bits(s.q_out).reshape(T, Hq, D)
     qo = r.q_out.reshape(T, Hq, D)
     H.assert_bits_equal(q[..., ~fpc], qo[..., ~fpc], "q_out pass-through columns")
-    H.assert_close_bf16(q[..., fpc], qo[..., fpc], "q_out", dtype=w.cache.dtype)
+    H.assert_close_bf16(q[..., fpc], qo[..., fpc], "q_out", dtype=w.cache.dtype, extra=eq)
     H.compare_paged_cache(w.cache, H.bits(s.storage), r.storage, r.written, w.layer_idx, fpc,
-                          "cache")
+                          "cache", k_extra=ek)
     return r
 
 
@@ -62,17 +84,34 @@ def test_per_head_norm_full_size(G):
     check_ragged(G, w, G.run_ragged(w))
 
 
-def _check_dual(G, w, s):
-    r = H.oracle_dual(w)
+def _check_dual(G, w, s, multiply_before_cast=True):
+    r = H.oracle_dual(w, multiply_before_cast=multiply_before_cast)
     assert int(s.err.item()) == r.err
     D = w.main_cache.head_dim
     allc = np.ones(D, bool)
-    for which, nq in (("main", w.main_q_heads), ("index", w.index_q_heads)):
+    bands = (("main", w.main_q_heads), ("index", w.index_q_heads))
+    x = H.values(H.bits(w.input), w.main_cache.dtype)
+    for k, (which, nq) in enumerate(bands if w.index_cache is not None else bands[:1]):
+        kv = getattr(w, f"{which}_cache")
+        eq = ek = None
+        if not multiply_before_cast:  # the reading's intermediate rounding (helpers.py)
+            cols = getattr(w, f"{which}_cols")
+            dt, eps = kv.dtype, getattr(w, f"{which}_eps")
+            gq, gk = (H.values(H.bits(g), dt) for g in w.gammas[2 * k:2 * k + 2])
+            eq = H.multiply_after_cast_slack(_head_rows(x, cols[0], nq, D), gq,
+                                             w.weight_offset, eps, dt, w.rope)
+            xk = (_head_rows(x, cols[1], kv.n_kv_heads, D) if cols[1] >= 0 else
+                  _slot_rows(kv, H.bits(kv.storage), kv.cache_lengths.tolist(), w.lengths,
+                             w.layer_idx))
+            ek = H.scatter_slots(kv, H.multiply_after_cast_slack(xk, gk, w.weight_offset, eps,
+                                                                 dt, w.rope),
+                                 kv.cache_lengths.tolist(), w.lengths, w.layer_idx)
         q = H.bits(getattr(s, f"q_{which}_out")).reshape(w.total_tokens, nq, D)
-        H.assert_close_bf16(q, r[f"q_{which}_out"].reshape(q.shape), f"q_{which}_out")
-        H.compare_paged_cache(getattr(w, f"{which}_cache"), H.bits(getattr(s, f"{which}_storage")),
+        H.assert_close_bf16(q, r[f"q_{which}_out"].reshape(q.shape), f"q_{which}_out",
+                            extra=eq)
+        H.compare_paged_cache(kv, H.bits(getattr(s, f"{which}_storage")),
                               r[f"{which}_storage"], r[f"{which}_written"], w.layer_idx, allc,
-                              f"{which} cache")
+                              f"{which} cache", k_extra=ek)
     return r
 
 

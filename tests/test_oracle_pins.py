@@ -554,3 +554,59 @@ def test_dual_band_geometry_mismatch_is_an_argument_error():
                     max_seq_len=16)
     w.index_cache.head_dim = 32
     assert H.oracle_dual(w).err == oracle.ERR_ARGS
+
+
+# ------------------------------------------------------------------- K updated in place --
+
+@pytest.mark.parametrize("single", [False, True])
+def test_k_in_place_on_a_cache_holding_the_inputs_k_is_the_store(single):
+    """fused_dual_qk_rms_norm_rope_ragged_paged (first paragraph): the key caches are
+    updated in place.  When the cache slots already hold the input's K and V rows (as the
+    projection would have stored them), normalising and rotating K where it lies must give
+    exactly what the store mode gives from the input: same Q outputs, same caches, every
+    other byte untouched."""
+    import copy
+    w = W.dual_band(113, lengths=[7, 12, 1], cache_lengths=[3, 40, 0], main_q_heads=4,
+                    main_kv_heads=2, index_q_heads=2, index_kv_heads=1, head_dim=64,
+                    main_page_size=16, index_page_size=8, rope_dim=32, theta=1e4,
+                    interleaved=False, max_seq_len=128, weight_offset=1.0, single=single)
+    store = H.oracle_dual(w)
+    assert store.err == 0
+    wi = copy.deepcopy(w)
+    D = w.main_cache.head_dim
+    for kv, cols in ((wi.main_cache, w.main_cols), (wi.index_cache, w.index_cols)):
+        if kv is None:
+            continue
+        Hk = kv.n_kv_heads
+        v6 = kv.view6()
+        for row, (page, slot) in enumerate(W.token_slots(kv, w.cache_lengths_of(kv),
+                                                          w.lengths)):
+            v6[page, 0, w.layer_idx, slot] = w.input[row, cols[1]:cols[1] + Hk * D].view(Hk, D)
+            if cols[2] >= 0:
+                v6[page, 1, w.layer_idx, slot] = \
+                    w.input[row, cols[2]:cols[2] + Hk * D].view(Hk, D)
+    wi.main_cols = (w.main_cols[0], -1, -1)
+    wi.index_cols = (w.index_cols[0], -1, -1)
+    inplace = H.oracle_dual(wi)
+    assert inplace.err == 0
+    for key in store:
+        if key != "err":
+            assert np.array_equal(inplace[key], store[key]), key
+
+
+def test_multiply_after_cast_with_unit_gamma_is_multiply_before_cast():
+    """multiply_before_cast has no definition on the pages (parity unpinned); the reading
+    taken (normalised value rounded to the element type, then scaled by gamma) must still
+    reduce to the plain op when gamma + weight_offset == 1 at position 0, where both orders
+    round the same normalised value once."""
+    w = W.ragged_store(114, lengths=[5], cache_lengths=[0], n_q_heads=2, n_kv_heads=1,
+                       head_dim=64, page_size=8, rope_dim=64, theta=1e4, interleaved=True,
+                       max_seq_len=8, norm=True, weight_offset=1.0, x_std=3.0)
+    w.q_gamma.zero_()
+    w.k_gamma.zero_()
+    w.cache.cache_lengths.zero_()
+    a = H.oracle_ragged_store(w, "bf16", True)
+    b = H.oracle_ragged_store(w, "bf16", False)
+    # row 0 sits at position 0: identity rotation; later rows rotate a rounded value
+    Hq, D = w.n_q_heads, w.cache.head_dim
+    assert np.array_equal(a.q_out.reshape(5, Hq * D)[0], b.q_out.reshape(5, Hq * D)[0])

@@ -304,6 +304,9 @@ class DualBand:
     def total_tokens(self) -> int:
         return self.input.shape[0]
 
+    def cache_lengths_of(self, kv: "PagedKV") -> List[int]:
+        return [int(x) for x in kv.cache_lengths]
+
 
 def dual_band(seed: int, *, lengths: List[int], cache_lengths: List[int], main_q_heads: int,
               main_kv_heads: int, index_q_heads: int, index_kv_heads: int, head_dim: int,
@@ -311,7 +314,11 @@ def dual_band(seed: int, *, lengths: List[int], cache_lengths: List[int], main_q
               interleaved: bool, max_seq_len: int, x_std: float = 1.0,
               main_eps: float = 1e-6, index_eps: float = 1e-6, weight_offset: float = 0.0,
               num_layers: int = 2, layer_idx: int = 1, dtype: str = "bf16",
-              name: str = "") -> DualBand:
+              k_in_place: bool = False, single: bool = False, name: str = "") -> DualBand:
+    """k_in_place: the bands' K heads are not read from the input but from the cache slots
+    the tokens map to (which hold N(0, x_std) K rows, as if the projection had stored them),
+    and V is not stored (the bands' column triples become (q_col, -1, -1)).  single: the
+    main band alone (index_cache, index outputs and the index gammas are None)."""
     gen = generator(seed)
     T, D = sum(lengths), head_dim
     qm, km, vm = 0, main_q_heads * D, (main_q_heads + main_kv_heads) * D
@@ -330,9 +337,41 @@ def dual_band(seed: int, *, lengths: List[int], cache_lengths: List[int], main_q
     gam = tuple(normal(gen, (D,), std=0.1, mean=1.0, dtype=dtype) for _ in range(4))
     q_main_out = random_bits(gen, T * main_q_heads * D, dtype).view(T, main_q_heads * D)
     q_index_out = random_bits(gen, T * index_q_heads * D, dtype).view(T, index_q_heads * D)
+    main_cols, index_cols = (qm, km, vm), (qi, ki, -1)
+    if k_in_place:
+        main_cols, index_cols = (qm, -1, -1), (qi, -1, -1)
+        for kv in (main, index):
+            fill_k_rows(gen, kv, cache_lengths, lengths, layer_idx, x_std)
+    if single:
+        index, index_q_heads, q_index_out = None, 0, None
+        gam = (gam[0], gam[1], None, None)
     return DualBand(inp, row_offsets(lengths), list(lengths), rope, layer_idx, main, index,
-                    (qm, km, vm), (qi, ki, -1), main_q_heads, index_q_heads, gam, main_eps,
+                    main_cols, index_cols, main_q_heads, index_q_heads, gam, main_eps,
                     index_eps, weight_offset, q_main_out, q_index_out, name)
+
+
+def token_slots(kv: PagedKV, cache_lengths: List[int], lengths: List[int]):
+    """(page, slot) of every new token, in row order (positions past the page table are
+    skipped)."""
+    out = []
+    for b, (c, n) in enumerate(zip(cache_lengths, lengths)):
+        for t in range(n):
+            pos = c + t
+            col = pos // kv.page_size
+            if col < kv.page_table.shape[1] and int(kv.page_table[b, col]) >= 0:
+                out.append((int(kv.page_table[b, col]), pos % kv.page_size))
+    return out
+
+
+def fill_k_rows(gen: torch.Generator, kv: PagedKV, cache_lengths: List[int],
+                lengths: List[int], layer_idx: int, std: float) -> None:
+    """Write N(0, std) K rows into the cache slots of the new tokens."""
+    slots = token_slots(kv, cache_lengths, lengths)
+    if not slots:
+        return
+    idx = torch.tensor(slots, dtype=torch.long)
+    kv.view6()[idx[:, 0], 0, layer_idx, idx[:, 1]] = normal(
+        gen, (len(slots), kv.n_kv_heads, kv.head_dim), std=std, dtype=kv.dtype)
 
 
 @dataclass
@@ -463,6 +502,20 @@ def per_head_norm(seed: int = 0) -> RaggedStore:
                         epsilon=1e-6, weight_offset=0.0, width=64,
                         name="per-head QK RMSNorm + RoPE + paged store: 64q/8kv heads, d128, "
                              "16384 tokens over 32 sequences")
+
+
+def dual_band_minimax_in_place(seed: int = 0) -> DualBand:
+    """dual_band_minimax with both key caches updated in place: K is read from the cache
+    slots (which hold N(0,1) K rows), V is not touched."""
+    gen = generator(seed)
+    lengths = lengths_with_total(gen, 64, 32768, 4096)
+    cls = uniform_ints(gen, 64, 0, 4096)
+    return dual_band(seed + 1, lengths=lengths, cache_lengths=cls, main_q_heads=64,
+                     main_kv_heads=8, index_q_heads=8, index_kv_heads=1, head_dim=128,
+                     main_page_size=128, index_page_size=64, rope_dim=64, theta=1e4,
+                     interleaved=True, max_seq_len=8192, k_in_place=True,
+                     name="dual-band fused launch, key caches updated in place: main "
+                          "64q/8kv + index 8q/1k, d128, partial RoPE 64, 32768 tokens")
 
 
 def dual_band_minimax(seed: int = 0) -> DualBand:
