@@ -94,9 +94,12 @@ def _load():
             _c_void_p, _c_void_p]
         lib.orc_kv_cache_radd.argtypes = [
             _i32, _c_void_p, _i64, _i32, P(_Paged), _c_void_p, _i32, _u32, _u32, _c_void_p]
+        lib.orc_matmul_fused_partial_rmsnorm.argtypes = [
+            _i32, _c_void_p, _c_void_p, _i64, _i32, _i32, _c_void_p, ctypes.c_double,
+            ctypes.c_double, _c_void_p, _i32, _c_void_p]
         for f in ("orc_rope_split_store_paged_ragged", "orc_fused_qk_rmsnorm_rope_paged",
                   "orc_fused_dual_qk_rmsnorm_rope_paged", "orc_qk_rope_bshd_continuous",
-                  "orc_kv_cache_radd"):
+                  "orc_kv_cache_radd", "orc_matmul_fused_partial_rmsnorm"):
             getattr(lib, f).restype = _u32
         lib.orc_decode.argtypes = [_i32, _c_void_p, _i64]
         lib.orc_decode.restype = ctypes.c_double
@@ -304,3 +307,16 @@ def encode(values, dtype: str) -> np.ndarray:
     for i in range(flat.size):
         lib.orc_encode(code, p, i, float(flat[i]))
     return out.reshape(v.shape)
+
+
+def matmul_fused_partial_rmsnorm(x, weight, gamma, epsilon, weight_offset, normed_output,
+                                 unnormed_output, dtype="bf16") -> int:
+    """MatmulFusedPartialRMSNorm (one input row): x [k], weight [n, k] (rows may be padded),
+    gamma [n_normed]; normed_output [n_normed] and unnormed_output [n - n_normed] are written
+    in place."""
+    n, k = weight.shape
+    nn = normed_output.shape[0]
+    assert unnormed_output.shape[0] == n - nn and x.shape[0] == k
+    return _load().orc_matmul_fused_partial_rmsnorm(
+        DTYPES[dtype], _ptr(x), _ptr(weight), _row_stride(weight), n, k, _ptr(gamma),
+        float(epsilon), float(weight_offset), _ptr(normed_output), nn, _ptr(unnormed_output))

@@ -414,3 +414,35 @@ uint32_t orc_kv_cache_radd(int32_t dtype, const void *a, int64_t a_row_stride,
   }
   return err;
 }
+
+/* ------------------------------------------------------- GEMV + partial RMSNorm (P5) -- */
+
+/* [P5] MatmulFusedPartialRMSNorm: y = x W^T for one input row (M = 1), W of shape (n, k);
+ * the first n_normed entries of y are RMS-normalised over those entries (epsilon inside
+ * the root) and scaled by gamma, the remaining n - n_normed pass through unchanged.
+ * weight_offset is accepted and not used, as the page states.  y is exact sums of
+ * products in double; every output is rounded once. */
+uint32_t orc_matmul_fused_partial_rmsnorm(int32_t dtype, const void *input, const void *weight,
+                                          int64_t weight_row_stride, int32_t n, int32_t k,
+                                          const void *gamma, double epsilon,
+                                          double weight_offset, void *normed_output,
+                                          int32_t n_normed, void *unnormed_output) {
+  (void)weight_offset; /* not consumed ([P5] Args) */
+  if (n < 0 || k < 0 || n_normed < 0 || n_normed > n || weight_row_stride < k) return ORC_ERR_ARGS;
+  const double eps = (double)(float)epsilon; /* a Float32 argument ([P5]) */
+  double *y = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  for (int64_t i = 0; i < n; ++i) {
+    double acc = 0.0;
+    for (int64_t j = 0; j < k; ++j)
+      acc += orc_decode(dtype, input, j) * orc_decode(dtype, weight, i * weight_row_stride + j);
+    y[i] = acc;
+  }
+  double ss = 0.0;
+  for (int64_t i = 0; i < n_normed; ++i) ss += y[i] * y[i];
+  const double r = n_normed > 0 ? 1.0 / sqrt(ss / n_normed + eps) : 0.0;
+  for (int64_t i = 0; i < n_normed; ++i)
+    orc_encode(dtype, normed_output, i, y[i] * r * orc_decode(dtype, gamma, i));
+  for (int64_t i = n_normed; i < n; ++i) orc_encode(dtype, unnormed_output, i - n_normed, y[i]);
+  free(y);
+  return 0;
+}

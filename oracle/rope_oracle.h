@@ -6,6 +6,7 @@
  *   "fused_dual_qk_rms_norm_rope_ragged_paged"     (per-head RMSNorm + RoPE, two caches)
  *   "generic_fused_qk_rope_bshd_continuous_batch"  (BSHD Q/K RoPE, continuous cache)
  *   "generic_kv_cache_radd_dispatch"               (in-place add into the K/V cache)
+ *   "MatmulFusedPartialRMSNorm"                    (GEMV + partial RMSNorm)
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the benchmark's
  * CPU-baseline leg may load this library.  It shares no code, header, table or helper with
@@ -122,6 +123,16 @@ uint32_t orc_kv_cache_radd(int32_t dtype, const void *a, int64_t a_row_stride,
                            int32_t total_tokens, orc_paged_cache *kv,
                            const uint32_t *input_row_offsets, int32_t batch,
                            uint32_t batch_offset, uint32_t layer_idx, uint8_t *written);
+
+/* "MatmulFusedPartialRMSNorm": y = x W^T (one input row, W of shape (n, k), row stride
+ * weight_row_stride); normed_output = the first n_normed entries of y RMS-normalised over
+ * themselves and scaled by gamma [n_normed]; unnormed_output = the other n - n_normed
+ * entries.  weight_offset is not used (as documented). */
+uint32_t orc_matmul_fused_partial_rmsnorm(int32_t dtype, const void *input, const void *weight,
+                                          int64_t weight_row_stride, int32_t n, int32_t k,
+                                          const void *gamma, double epsilon,
+                                          double weight_offset, void *normed_output,
+                                          int32_t n_normed, void *unnormed_output);
 
 /* element codecs, exported so that the self-tests can pin them */
 double orc_decode(int32_t dtype, const void *base, int64_t i);

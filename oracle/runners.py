@@ -115,3 +115,11 @@ def oracle_radd(w: "W.Radd", dtype: str = "bf16") -> OracleResult:
     err = oracle.kv_cache_radd(bits(w.a), oracle_paged(w.cache, store), bits(w.offsets),
                                w.batch_offset, w.layer_idx, written, dtype)
     return OracleResult(storage=store, written=written, err=err)
+
+
+def oracle_gemv(w: "W.GemvNorm", dtype: str = "bf16") -> OracleResult:
+    normed, unnormed = bits(w.normed_output), bits(w.unnormed_output)
+    err = oracle.matmul_fused_partial_rmsnorm(bits(w.x), bits(w.weight), bits(w.gamma),
+                                              w.epsilon, w.weight_offset, normed, unnormed,
+                                              dtype)
+    return OracleResult(normed=normed, unnormed=unnormed, err=err)

@@ -14,7 +14,7 @@ import workloads as W
 
 from oracle.runners import (bits, oracle_rope, oracle_paged, oracle_cont,  # noqa: F401
                             OracleResult, oracle_ragged_store, oracle_dual, oracle_bshd,
-                            oracle_radd)
+                            oracle_radd, oracle_gemv)
 
 
 def values(b: np.ndarray, dtype: str) -> np.ndarray:

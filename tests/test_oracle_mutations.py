@@ -4,7 +4,8 @@ on the CPU, makes the pin suite fail.
 Each mutant is a one-line edit of rope_oracle.c (a flipped sign, swapped cos/sin, a wrong
 pair partner, a dropped cache length, epsilon outside the root, a sum instead of a mean, a
 dropped weight_offset, a shifted slot, swapped K/V halves, an off-by-one valid length, the
-wrong rotated columns).  The copy is built in a temporary directory and the pin suite runs
+wrong rotated columns, and in the GEMV + partial RMSNorm: epsilon outside the root, the
+mean over every column, the norm over the tail, a consumed weight_offset).  The copy is built in a temporary directory and the pin suite runs
 against it in a subprocess; the test passes when that run fails.
 """
 import os
@@ -41,6 +42,19 @@ MUTANTS = {
     "partial rope on the leading columns": (
         "return rope->rope_col_offset < 0 ? head_dim - rope->rope_dim : rope->rope_col_offset;",
         "return rope->rope_col_offset < 0 ? 0 : rope->rope_col_offset;"),
+    "gemv epsilon outside the root": (
+        "const double r = n_normed > 0 ? 1.0 / sqrt(ss / n_normed + eps) : 0.0;",
+        "const double r = n_normed > 0 ? 1.0 / sqrt(ss / n_normed) + eps : 0.0;"),
+    "gemv mean over every column": (
+        "const double r = n_normed > 0 ? 1.0 / sqrt(ss / n_normed + eps) : 0.0;",
+        "const double r = n_normed > 0 ? 1.0 / sqrt(ss / n + eps) : 0.0;"),
+    "gemv norm taken over the tail": (
+        "for (int64_t i = 0; i < n_normed; ++i) ss += y[i] * y[i];",
+        "for (int64_t i = n - n_normed; i < n; ++i) ss += y[i] * y[i];"),
+    "gemv weight_offset consumed": (
+        "orc_encode(dtype, normed_output, i, y[i] * r * orc_decode(dtype, gamma, i));",
+        "orc_encode(dtype, normed_output, i, y[i] * r * (orc_decode(dtype, gamma, i) + "
+        "weight_offset));"),
 }
 
 

@@ -610,3 +610,68 @@ def test_multiply_after_cast_with_unit_gamma_is_multiply_before_cast():
     # row 0 sits at position 0: identity rotation; later rows rotate a rounded value
     Hq, D = w.n_q_heads, w.cache.head_dim
     assert np.array_equal(a.q_out.reshape(5, Hq * D)[0], b.q_out.reshape(5, Hq * D)[0])
+
+
+# ------------------------------------------------ GEMV + partial RMSNorm (P5) ----------
+
+def _gemv(n, k, n_normed, dtype="f32", seed=120, **kw):
+    return W.gemv_norm(seed, n=n, k=k, n_normed=n_normed, dtype=dtype, **kw)
+
+
+def _vals(a, dtype):
+    return H.values(a, dtype)
+
+
+def test_gemv_pass_through_is_the_rounded_matmul():
+    # MatmulFusedPartialRMSNorm: the columns after n_normed are y = x W^T unchanged; numpy's
+    # float64 matmul of the decoded inputs is the exact product up to its summation order
+    w = _gemv(37, 300, 5, dtype="bf16", row_pad=8)
+    r = H.oracle_gemv(w, "bf16")
+    assert r.err == 0
+    x = w.x.double().numpy()
+    y = w.weight.double().numpy() @ x
+    assert _within_half_ulp(_vals(r.unnormed, "bf16"), y[5:])
+
+
+def test_gemv_normed_rms_closed_form():
+    # with gamma = g constant: rms(normed) = |g| sqrt(ms / (ms + eps)) over the normed part
+    eps, g = 0.25, 1.5
+    w = _gemv(24, 96, 16, epsilon=eps)
+    w.gamma.fill_(g)
+    r = H.oracle_gemv(w, "f32")
+    y = w.weight.double().numpy() @ w.x.double().numpy()
+    ms = (y[:16] ** 2).mean()
+    got = r.normed.astype(np.float64)
+    np.testing.assert_allclose(np.sqrt((got ** 2).mean()), g * np.sqrt(ms / (ms + eps)),
+                               rtol=1e-6)
+    # the direction of the normed part is y's
+    np.testing.assert_allclose(got / np.linalg.norm(got), y[:16] / np.linalg.norm(y[:16]),
+                               rtol=1e-5, atol=1e-7)
+
+
+def test_gemv_scale_invariance_and_gamma():
+    # eps = 0: scaling x by 2 (exact) leaves the normed part unchanged bit for bit and doubles
+    # the pass-through part; gamma scales the normed part elementwise
+    w = _gemv(20, 64, 12, dtype="bf16", epsilon=0.0)
+    a = H.oracle_gemv(w, "bf16")
+    w2 = W.GemvNorm(w.x * 2, w.weight, w.gamma, 0.0, 0.0, w.normed_output,
+                    w.unnormed_output)
+    b = H.oracle_gemv(w2, "bf16")
+    assert np.array_equal(a.normed, b.normed)
+    np.testing.assert_array_equal(_vals(b.unnormed, "bf16"), 2 * _vals(a.unnormed, "bf16"))
+    w3 = W.GemvNorm(w.x, w.weight, w.gamma * 4, 0.0, 0.0, w.normed_output, w.unnormed_output)
+    c = H.oracle_gemv(w3, "bf16")
+    np.testing.assert_array_equal(_vals(c.normed, "bf16"), 4 * _vals(a.normed, "bf16"))
+
+
+def test_gemv_weight_offset_is_not_consumed_and_partitions_agree():
+    w = _gemv(30, 128, 10, dtype="bf16")
+    a = H.oracle_gemv(w, "bf16")
+    w.weight_offset = 3.0
+    b = H.oracle_gemv(w, "bf16")
+    assert np.array_equal(a.normed, b.normed) and np.array_equal(a.unnormed, b.unnormed)
+    # no normed columns: every column passes through; the 20 trailing ones are a's
+    w0 = W.GemvNorm(w.x, w.weight, w.gamma[:0], w.epsilon, 0.0, w.normed_output[:0],
+                    W.random_bits(W.generator(1), 30, "bf16"))
+    z = H.oracle_gemv(w0, "bf16")
+    assert np.array_equal(z.unnormed[10:], a.unnormed)

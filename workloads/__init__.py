@@ -542,3 +542,55 @@ def radd_minimax(seed: int = 0) -> Radd:
     return radd(seed + 1, lengths=lengths, cache_lengths=cls, n_kv_heads=8, head_dim=128,
                 page_size=128, batch_offset=0,
                 name="kv_cache_radd: bf16 [32768, 2048] into the main cache, page 128")
+
+
+# ------------------------------------------------------- GEMV + partial RMSNorm inputs --
+
+@dataclass
+class GemvNorm:
+    """One input row x [k], weight W [n, k] (y = x W^T), gamma [n_normed]; the outputs start
+    as random-bit sentinels."""
+    x: torch.Tensor
+    weight: torch.Tensor
+    gamma: torch.Tensor
+    epsilon: float
+    weight_offset: float
+    normed_output: torch.Tensor
+    unnormed_output: torch.Tensor
+    name: str = ""
+
+    @property
+    def n(self) -> int:
+        return self.weight.shape[0]
+
+    @property
+    def k(self) -> int:
+        return self.weight.shape[1]
+
+    @property
+    def n_normed(self) -> int:
+        return self.normed_output.shape[0]
+
+
+def gemv_norm(seed: int, *, n: int, k: int, n_normed: int, epsilon: float = 1e-6,
+              weight_offset: float = 0.0, dtype: str = "bf16", row_pad: int = 0,
+              name: str = "") -> GemvNorm:
+    """x ~ N(0,1), W ~ N(0, 1/k) so that y ~ N(0,1), gamma ~ N(1, 0.1)."""
+    gen = generator(seed)
+    x = normal(gen, (k,), dtype=dtype)
+    w = normal(gen, (n, k + row_pad), std=k ** -0.5, dtype=dtype)
+    if row_pad:
+        w = w[:, :k]
+    gamma = normal(gen, (n_normed,), std=0.1, mean=1.0, dtype=dtype)
+    normed = random_bits(gen, n_normed, dtype)
+    unnormed = random_bits(gen, n - n_normed, dtype)
+    return GemvNorm(x, w, gamma, epsilon, weight_offset, normed, unnormed, name)
+
+
+def mla_kv_a_proj(seed: int = 0) -> GemvNorm:
+    """The decode-time producer of a latent-attention KV cache entry: hidden 7168 projected
+    to a 512-wide latent (RMS-normalised) and a 64-wide rotary key part (passed through),
+    one token."""
+    return gemv_norm(seed, n=576, k=7168, n_normed=512, epsilon=1e-6,
+                     name="GEMV + partial RMSNorm: x [7168] @ W^T [576, 7168], first 512 "
+                          "normed, last 64 passed through")
