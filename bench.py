@@ -188,6 +188,12 @@ def bytes_dual(w) -> int:
         w.rope, positions_ragged(w.lengths, w.main_cache.cache_lengths.tolist()))
 
 
+def bytes_gemv(w) -> int:
+    """W read + x read + gamma read + the n outputs written."""
+    eb = w.weight.element_size()
+    return (w.n * w.k + w.k + w.n_normed + w.n) * eb
+
+
 def bytes_radd(w) -> int:
     """a read + cache rows read + cache rows written."""
     return w.a.shape[0] * 3 * w.a.shape[1] * w.a.element_size()
@@ -213,7 +219,10 @@ WORKLOADS = {
     "dual_band_minimax_in_place": "fused_dual_qk_rmsnorm_rope_paged",
     "radd_minimax": "kv_cache_radd",
     "decode_bshd": "qk_rope_bshd_continuous",
+    "mla_kv_a_proj": "matmul_fused_partial_rmsnorm",
 }
+# copies of a workload the steps rotate over: enough that their inputs exceed L2 (126 MB)
+REPLICAS_OF = {"mla_kv_a_proj": 24}
 
 
 class Case:
@@ -230,7 +239,7 @@ def make_workload(name, seed):
             "dual_band_minimax": W.dual_band_minimax,
             "dual_band_minimax_in_place": W.dual_band_minimax_in_place,
             "radd_minimax": W.radd_minimax,
-            "decode_bshd": W.decode_bshd}[name](seed)
+            "decode_bshd": W.decode_bshd, "mla_kv_a_proj": W.mla_kv_a_proj}[name](seed)
 
 
 def make_case(name, seed, dev, w=None, sched=True):
@@ -411,6 +420,30 @@ def make_case(name, seed, dev, w=None, sched=True):
         c.config = {"q_proj": list(w.q_proj.shape), "n_kv_heads": kv.n_kv_heads,
                     "cache": [kv.num_slots, kv.max_seq_len], "rope": "interleaved, freqs bf16"}
         c.workload = w
+    elif name == "mla_kv_a_proj":
+        w = w or make_workload(name, seed)
+        x, wt, g = d(w.x), d(w.weight), d(w.gamma)
+        no, uo = d(w.normed_output), d(w.unnormed_output)
+        c.ws = rs.gemv_workspace(w.n_normed, dev)
+        args = (x.data_ptr(), wt.data_ptr(), wt.stride(0), w.n, w.k, 1, g.data_ptr(),
+                ctypes.c_float(w.epsilon), ctypes.c_float(w.weight_offset), no.data_ptr(),
+                w.n_normed, uo.data_ptr(), 0, c.err.data_ptr(), c.ws.data_ptr(),
+                c.ws.numel() * 4, stream.cuda_stream)
+        c.step = bind(lib.matmul_fused_partial_rmsnorm, args, c.entry_point)
+
+        def call():
+            rs.matmul_fused_partial_rmsnorm(x, wt, g, w.epsilon, w.weight_offset, no, uo, c.ws,
+                                            err_word=c.err)
+        c.call = call
+        c.tokens = 1
+        c.alg_bytes = bytes_gemv(w)
+        c.e2e_in = [(pinned(w.x), x)]
+        c.e2e_out = [(no, torch.empty(no.shape, dtype=no.dtype).pin_memory()),
+                     (uo, torch.empty(uo.shape, dtype=uo.dtype).pin_memory())]
+        c.outputs = [no, uo]
+        c.config = {"n": w.n, "k": w.k, "n_normed": w.n_normed, "weight_bytes":
+                    w.weight.numel() * w.weight.element_size()}
+        c.workload = w
     else:
         raise ValueError(name)
     c.keep = keep
@@ -526,8 +559,8 @@ def run_ours(args):
     use_sched = args.schedule == "claimed"
     # this rank's replica: its own seeded batch, staged REPLICAS times
     w = make_workload(args.workload, 1000 * rank)
-    cases = [make_case(args.workload, 1000 * rank, dev, w, use_sched)
-             for _ in range(REPLICAS)]
+    n_rep = REPLICAS_OF.get(args.workload, REPLICAS)
+    cases = [make_case(args.workload, 1000 * rank, dev, w, use_sched) for _ in range(n_rep)]
     case = cases[0]
     stream = torch.cuda.current_stream()
     props = torch.cuda.get_device_properties(dev)
@@ -537,7 +570,7 @@ def run_ours(args):
 
     W_ = max(3, args.warmup)
     for i in range(W_):
-        steps[i % REPLICAS]()
+        steps[i % n_rep]()
     torch.cuda.synchronize()
     if args.workload != "radd_minimax":   # radd accumulates: its data stays valid anyway
         assert all(int(c.err.item()) == 0 for c in cases), "device error bits set"
@@ -587,7 +620,7 @@ def run_ours(args):
         "data": "synthetic (seeded, shapes of the named workload)",
         "config": dict({"workload": case.workload.name, "entry_point": case.entry_point,
                         "tokens_per_rank": case.tokens, "cache_dtype": "bf16",
-                        "l2": f"inputs larger than L2: {REPLICAS} rotating copies of the "
+                        "l2": f"inputs larger than L2: {n_rep} rotating copies of the "
                               f"workload, launched back to back",
                         "overlap": OVERLAP_NAMES[args.overlap],
                         "schedule": "claimed tail (scheduling workspace)" if use_sched
@@ -626,7 +659,8 @@ KERNELS = {"llama3_8b_prefill": "banded_store_kernel<bf16, head_dim 128, no norm
            "dual_band_minimax_in_place":
                "banded_store_kernel<bf16, head_dim 128, rmsnorm> (two bands, K in place)",
            "radd_minimax": "radd_kernel<bf16, head_dim 128>",
-           "decode_bshd": "bshd_rope_kernel<bf16, head_dim 128>"}
+           "decode_bshd": "bshd_rope_kernel<bf16, head_dim 128>",
+           "mla_kv_a_proj": "gemv_norm_kernel<bf16, 4 rows per CTA>"}
 
 
 def summarize(case, sec, peak):
@@ -647,13 +681,14 @@ def launch_modes(torch, dev, stream, args, w, peak, reps=300):
     import rope_paged_kv_b200 as rs
     out = {}
     for use_sched in (True, False):
-        cases = [make_case(args.workload, 0, dev, w, use_sched) for _ in range(REPLICAS)]
+        cases = [make_case(args.workload, 0, dev, w, use_sched)
+                 for _ in range(REPLICAS_OF.get(args.workload, REPLICAS))]
         steps = [c.step for c in cases]
         tag = "claimed" if use_sched else "static"
         for mode in (0, 1, 2):
             rs.set_launch_overlap(mode)
             for i in range(6):
-                steps[i % REPLICAS]()
+                steps[i % len(steps)]()
             sec = time_steps(torch, steps, reps, stream) / reps / 1e3
             out[f"{tag}/{OVERLAP_NAMES[mode]}"] = summarize(cases[0], sec, peak)["us_per_launch"]
         rs.set_launch_overlap(0)
@@ -673,10 +708,11 @@ def run_entry_points(torch, dev, stream, headline, peak, use_sched, reps=30):
         if name == headline:
             continue
         w = make_workload(name, 0)
-        cases = [make_case(name, 0, dev, w, use_sched) for _ in range(REPLICAS)]
+        cases = [make_case(name, 0, dev, w, use_sched)
+                 for _ in range(REPLICAS_OF.get(name, REPLICAS))]
         steps = [c.step for c in cases]
         for i in range(3):
-            steps[i % REPLICAS]()
+            steps[i % len(steps)]()
         sec = time_steps(torch, steps, reps, stream) / reps / 1e3
         out[name] = summarize(cases[0], sec, peak)
         if name == "decode_bshd":

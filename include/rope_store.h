@@ -267,6 +267,34 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
                             int32_t batch, uint32_t batch_offset, uint32_t layer_idx,
                             uint32_t *err_word, uint32_t *sched, rope_stream_t stream);
 
+/* matmul_fused_partial_rmsnorm -- MatmulFusedPartialRMSNorm page (description, execute,
+ * Args): the one-row GEMV y = input W^T (M = 1) fused with an RMSNorm over its first
+ * n_normed entries.
+ *   input [k], weight [n, k] row-major with row stride weight_row_stride (elements) -- the
+ *   page's default transpose_b = True; transpose_b = 0 (weight stored [k, n]) returns
+ *   ROPE_ERR_UNSUPPORTED.  gamma [n_normed].
+ *   normed_output [n_normed] = y[i] * rsqrt(mean(y[0..n_normed)^2) + epsilon) * gamma[i];
+ *   unnormed_output [n - n_normed] = y[n_normed..n) unchanged.
+ *   weight_offset is accepted and not used, as the page states.
+ *   dtype (rope_dtype_t) is the element type of every tensor; y is accumulated in float32
+ *   and each output rounded once.  k * element size must be a multiple of 16 bytes, and
+ *   input / weight / workspace 16-byte aligned.
+ *   err_word: as for the other calls (only ROPE_DEVERR_TIMEOUT can occur here).
+ *   workspace: device memory of at least ROPE_GEMV_WORKSPACE_BYTES(n_normed) bytes (may be
+ *   NULL when n_normed == 0) whose first word must be zero before the first call that uses
+ *   it; every call leaves it zero.  It holds the float32 entries to be normalised until the
+ *   last CTA normalises them.  Calls that can run at the same time need separate
+ *   workspaces. */
+#define ROPE_GEMV_WORKSPACE_BYTES(n_normed) (16 + 4 * (int64_t)(n_normed))
+rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight,
+                                           int64_t weight_row_stride, int32_t n, int32_t k,
+                                           int32_t transpose_b, const void *gamma,
+                                           float epsilon, float weight_offset,
+                                           void *normed_output, int32_t n_normed,
+                                           void *unnormed_output, int32_t dtype,
+                                           uint32_t *err_word, void *workspace,
+                                           int64_t workspace_bytes, rope_stream_t stream);
+
 /* rope_split_store_paged_ragged_noalloc -- rope_split_store_paged_ragged with the
  * claimed-tail schedule, for callers that cannot allocate device memory: for example a
  * plug-in inside an engine that hands out all device memory from its own pool and allows no

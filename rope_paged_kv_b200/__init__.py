@@ -104,12 +104,16 @@ _lib.kv_cache_radd.argtypes = [
 _lib.rope_split_store_paged_ragged_noalloc.argtypes = [
     _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp,
     _vp]
+_lib.matmul_fused_partial_rmsnorm.argtypes = [
+    _vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _f32, _vp, _i32, _vp, _i32, _vp, _vp, _i64,
+    _vp]
 _lib.rope_set_launch_overlap.argtypes = [_i32]
 _lib.rope_get_launch_overlap.argtypes = []
 _lib.rope_get_launch_overlap.restype = _i32
 for _f in ("rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
            "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd",
-           "rope_set_launch_overlap", "rope_split_store_paged_ragged_noalloc"):
+           "rope_set_launch_overlap", "rope_split_store_paged_ragged_noalloc",
+           "matmul_fused_partial_rmsnorm"):
     getattr(_lib, _f).restype = ctypes.c_int
 _lib.rope_status_string.argtypes = [ctypes.c_int]
 _lib.rope_status_string.restype = ctypes.c_char_p
@@ -346,6 +350,35 @@ def kv_cache_radd(a, kv: PagedCache, input_row_offsets, batch_offset, layer_idx,
         a.data_ptr(), _row_stride(a), a.shape[0], ctypes.byref(c), offs.data_ptr(),
         offs.shape[0] - 1, batch_offset, layer_idx, _ptr(err_word), _sched(sched),
         _stream(stream)), "kv_cache_radd")
+
+
+def gemv_workspace_bytes(n_normed: int) -> int:
+    return 16 + 4 * int(n_normed)
+
+
+def gemv_workspace(n_normed: int, device=None) -> torch.Tensor:
+    """A zeroed workspace for matmul_fused_partial_rmsnorm (16-byte aligned)."""
+    return torch.zeros(gemv_workspace_bytes(n_normed) // 4, dtype=torch.int32,
+                       device=device if device is not None else torch.cuda.current_device())
+
+
+def matmul_fused_partial_rmsnorm(input, weight, gamma, epsilon, weight_offset, normed_output,
+                                 unnormed_output, workspace=None, stream=None,
+                                 err_word=None) -> None:
+    """y = input @ weight.T (input [k], weight [n, k]); normed_output [n_normed] gets the RMS
+    normalised first entries times gamma, unnormed_output [n - n_normed] the rest."""
+    n, k = weight.shape
+    nn = normed_output.shape[0]
+    if unnormed_output.shape[0] != n - nn or input.shape[-1] != k:
+        raise ValueError("output sizes must split n; input must have k entries")
+    dtype = _DTYPE_CODE[weight.dtype]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.matmul_fused_partial_rmsnorm(
+        input.data_ptr(), weight.data_ptr(), _row_stride(weight), n, k, 1,
+        gamma.data_ptr() if nn else None, epsilon, weight_offset,
+        normed_output.data_ptr() if nn else None, nn,
+        unnormed_output.data_ptr() if n > nn else None, dtype, _ptr(err_word), _ptr(workspace),
+        ws_bytes, _stream(stream)), "matmul_fused_partial_rmsnorm")
 
 
 def raw_library() -> ctypes.CDLL:

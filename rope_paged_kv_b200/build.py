@@ -13,7 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librope_store.so")
 SOURCES = [os.path.join(CSRC, "rope_store.cu")]
-HEADERS = ["device_utils.cuh", "pipeline.cuh", "common.cuh", "banded.cuh", "bshd.cuh", "radd.cuh"]
+HEADERS = ["device_utils.cuh", "pipeline.cuh", "common.cuh", "banded.cuh", "bshd.cuh", "radd.cuh",
+           "gemv_norm.cuh"]
 DEPS = SOURCES + [os.path.join(CSRC, h) for h in HEADERS] + [
                   os.path.join(ROOT, "include", "rope_store.h")]
 

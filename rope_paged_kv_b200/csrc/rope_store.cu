@@ -5,10 +5,13 @@
 //               CTAs, a producer warp bulk-copying token rows into a shared-memory ring,
 //               eight consumer warps rotating / normalising and storing;
 //   radd.cuh    in-place cache add on the same staging scheme;
-//   bshd.cuh    decode-shaped BSHD RoPE with in-place K, one CTA per token.
+//   bshd.cuh    decode-shaped BSHD RoPE with in-place K, one CTA per token;
+//   gemv_norm.cuh  one-row GEMV + partial RMSNorm, a few rows of W per CTA, the last CTA
+//               normalising.
 #include "../../include/rope_store.h"
 #include "banded.cuh"
 #include "bshd.cuh"
+#include "gemv_norm.cuh"
 #include "radd.cuh"
 
 #include <cuda_runtime.h>
@@ -433,6 +436,33 @@ static rope_status_t launch_radd_d(int D, const RaddParams &p, size_t smem, cuda
   return ROPE_ERR_UNSUPPORTED;
 }
 
+// ------------------------------------------------------------- GEMV + partial RMSNorm --
+
+constexpr int kGemvSmemMax = 200 << 10;  // shared memory a staged GEMV CTA may take
+
+template <typename T, int R>
+static rope_status_t launch_gemv_r(const GemvParams &p, cudaStream_t st) {
+  const int grid = (p.n + R - 1) / R;
+  const size_t smem = (size_t)p.row_bytes * (R + 1);
+  if (smem <= (size_t)kGemvSmemMax) {  // x and the CTA's rows fit: bulk-copy them
+    static ShapeCache cache;
+    auto kern = gemv_norm_kernel<T, R, true>;
+    if (resident_ctas(kern, kGemvThreads, smem, cache) <= 0) return ROPE_ERR_UNSUPPORTED;
+    return launch(kern, grid, kGemvThreads, smem, st, p);
+  }
+  return launch(gemv_norm_kernel<T, R, false>, grid, kGemvThreads, 0, st, p);
+}
+
+// rows per CTA: the fewest that keep the grid within one CTA per SM (at most 8)
+template <typename T>
+static rope_status_t launch_gemv_t(const GemvParams &p, cudaStream_t st) {
+  const int sms = sm_count() > 0 ? sm_count() : 1;
+  if (p.n <= sms) return launch_gemv_r<T, 1>(p, st);
+  if (p.n <= 2 * sms) return launch_gemv_r<T, 2>(p, st);
+  if (p.n <= 4 * sms) return launch_gemv_r<T, 4>(p, st);
+  return launch_gemv_r<T, 8>(p, st);
+}
+
 // ------------------------------------------------------- allocation-free entry point --
 // Scheduling workspace of rope_split_store_paged_ragged_noalloc.  Every device that loads
 // the library holds one copy of this array until the process exits, and every call of that
@@ -700,6 +730,52 @@ rope_status_t rope_split_store_paged_ragged_noalloc(
   return rope_split_store_paged_ragged(qkv, qkv_row_stride, total_tokens, n_q_heads,
                                        input_row_offsets, batch, freqs, kv, layer_idx, q_out,
                                        q_out_row_stride, err_word, scratch, stream);
+}
+
+rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight,
+                                           int64_t weight_row_stride, int32_t n, int32_t k,
+                                           int32_t transpose_b, const void *gamma,
+                                           float epsilon, float weight_offset,
+                                           void *normed_output, int32_t n_normed,
+                                           void *unnormed_output, int32_t dtype,
+                                           uint32_t *err_word, void *workspace,
+                                           int64_t workspace_bytes, rope_stream_t stream) {
+  (void)weight_offset;  // accepted for a uniform signature; not used by this operation
+  if (n < 0 || k < 0 || n_normed < 0 || n_normed > n) return ROPE_ERR_INVALID_ARG;
+  if (n == 0) return ROPE_OK;  // no output: nothing is read or written
+  if (transpose_b == 0) return ROPE_ERR_UNSUPPORTED;
+  const int eb = elem_bytes(dtype);
+  if (eb == 0) return ROPE_ERR_UNSUPPORTED;
+  if (weight == nullptr || weight_row_stride < k || (k > 0 && input == nullptr) ||
+      (n_normed > 0 && (gamma == nullptr || normed_output == nullptr || workspace == nullptr)) ||
+      (n > n_normed && unnormed_output == nullptr))
+    return ROPE_ERR_INVALID_ARG;
+  if (n_normed > 0 && workspace_bytes < ROPE_GEMV_WORKSPACE_BYTES(n_normed))
+    return ROPE_ERR_INVALID_ARG;
+  if ((k * eb) % 16 || !aligned16(weight) || !stride16(weight_row_stride, eb) ||
+      (k > 0 && !aligned16(input)) || (n_normed > 0 && !aligned16(workspace)))
+    return ROPE_ERR_UNSUPPORTED;
+  GemvParams p{};
+  p.x = input;
+  p.w = weight;
+  p.w_stride = weight_row_stride;
+  p.n = n;
+  p.k = k;
+  p.n_normed = n_normed;
+  p.gamma = gamma;
+  p.eps = epsilon;
+  p.normed = normed_output;
+  p.unnormed = unnormed_output;
+  p.count = static_cast<uint32_t *>(workspace);
+  p.ws = workspace ? reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + 16)
+                   : nullptr;
+  p.err = err_word;
+  p.row_bytes = (int32_t)round_up((int64_t)k * eb, 16);
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype == ROPE_DTYPE_BF16) return launch_gemv_t<__nv_bfloat16>(p, st);
+  if (dtype == ROPE_DTYPE_F16) return launch_gemv_t<__half>(p, st);
+  return launch_gemv_t<float>(p, st);
 }
 
 rope_status_t rope_set_launch_overlap(int32_t mode) {

@@ -153,3 +153,20 @@ def test_launch_overlap_mode(rs):
         assert lib.rope_get_launch_overlap() == rs.OVERLAP_PDL
     finally:
         lib.rope_set_launch_overlap(before)
+
+
+def test_gemv_host_checks_need_no_gpu(rs):
+    lib = rs.raw_library()
+    fake = 1 << 20
+    call = lib.matmul_fused_partial_rmsnorm
+    args = [fake, fake, 64, 8, 64, 1, fake, 1e-6, 0.0, fake, 8, None, 0, None, fake, 48, None]
+    bad = list(args); bad[10] = 9          # n_normed > n
+    assert call(*bad) == rs.ERR_INVALID_ARG
+    bad = list(args); bad[5] = 0           # weight stored [k, n] (transpose_b = False)
+    assert call(*bad) == rs.ERR_UNSUPPORTED
+    bad = list(args); bad[3] = 0; bad[10] = 0  # no output at all: OK without a launch
+    assert call(*bad) == rs.OK
+    bad = list(args); bad[15] = 16         # workspace smaller than ROPE_GEMV_WORKSPACE_BYTES
+    assert call(*bad) == rs.ERR_INVALID_ARG
+    bad = list(args); bad[12] = 7          # unknown element type
+    assert call(*bad) == rs.ERR_UNSUPPORTED
