@@ -125,29 +125,31 @@ __global__ void __launch_bounds__(kGemvThreads)
         }
       }
     }
-  } else
-  for (int c0 = tid; c0 < chunks; c0 += kGemvThreads * kGemvUnroll) {
-    uint4 xv[kGemvUnroll], wv[kGemvUnroll][R];
+  } else {  // (braced: an unbraced statement here was compiled as if the rest of the
+           // kernel belonged to the discarded branch)
+    for (int c0 = tid; c0 < chunks; c0 += kGemvThreads * kGemvUnroll) {
+      uint4 xv[kGemvUnroll], wv[kGemvUnroll][R];
 #pragma unroll
-    for (int u = 0; u < kGemvUnroll; ++u) {
-      const int c = c0 + u * kGemvThreads;
-      xv[u] = c < chunks ? ld_plain(x + (int64_t)c * N) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < kGemvUnroll; ++u) {
+        const int c = c0 + u * kGemvThreads;
+        xv[u] = c < chunks ? ld_plain(x + (int64_t)c * N) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int r = 0; r < R; ++r)
-        wv[u][r] = (c < chunks && row0 + r < p.n)
-                       ? ld_stream(w + (int64_t)(row0 + r) * p.w_stride + (int64_t)c * N)
-                       : make_uint4(0, 0, 0, 0);
-    }
+        for (int r = 0; r < R; ++r)
+          wv[u][r] = (c < chunks && row0 + r < p.n)
+                         ? ld_stream(w + (int64_t)(row0 + r) * p.w_stride + (int64_t)c * N)
+                         : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (int u = 0; u < kGemvUnroll; ++u) {
-      float xf[N];
-      VT::widen(xv[u], xf);
+      for (int u = 0; u < kGemvUnroll; ++u) {
+        float xf[N];
+        VT::widen(xv[u], xf);
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        float wf[N];
-        VT::widen(wv[u][r], wf);
+        for (int r = 0; r < R; ++r) {
+          float wf[N];
+          VT::widen(wv[u][r], wf);
 #pragma unroll
-        for (int e = 0; e < N; ++e) acc[r] = fmaf(xf[e], wf[e], acc[r]);
+          for (int e = 0; e < N; ++e) acc[r] = fmaf(xf[e], wf[e], acc[r]);
+        }
       }
     }
   }
