@@ -293,7 +293,7 @@ def make_case(name, seed, dev, w=None, sched=True):
         if w.q_gamma is None:
             args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
                     offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), w.layer_idx,
-                    q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(), sched_ptr,
+                    q_out.data_ptr(), q_out.stride(0), -1, c.err.data_ptr(), sched_ptr,
                     stream.cuda_stream)
             c.step = bind(lib.rope_split_store_paged_ragged, args, c.entry_point)
 

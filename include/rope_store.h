@@ -189,16 +189,19 @@ typedef struct {
  *   input_row_offsets [batch + 1]: sequence b owns rows [offs[b], offs[b+1]).
  *   Row r of sequence b sits at position p = kv->cache_lengths[b] + (r - offs[b]).
  *   Q heads are rotated with freqs_cis row p and written to q_out [total_tokens, n_q_heads *
- *   head_dim] (row stride q_out_row_stride); K heads are rotated and V heads copied into the
- *   cache of layer layer_idx at position p.  kv->v must not be NULL. */
+ *   head_dim] (row stride q_out_row_stride, in q_out elements); K heads are rotated and V
+ *   heads copied into the cache of layer layer_idx at position p.  kv->v must not be NULL.
+ *   q_out_dtype (rope_dtype_t; < 0: the cache's element type) is the element type of q_out
+ *   (the page's q_out_dtype parameter, which defaults to dtype): rotated values are rounded
+ *   once into it and unrotated columns converted exactly or rounded once. */
 rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_stride,
                                             int32_t total_tokens, int32_t n_q_heads,
                                             const uint32_t *input_row_offsets, int32_t batch,
                                             const rope_freqs_t *freqs,
                                             const rope_paged_cache_t *kv, uint32_t layer_idx,
                                             void *q_out, int64_t q_out_row_stride,
-                                            uint32_t *err_word, uint32_t *sched,
-                                            rope_stream_t stream);
+                                            int32_t q_out_dtype, uint32_t *err_word,
+                                            uint32_t *sched, rope_stream_t stream);
 
 /* fused_qk_rmsnorm_rope_paged -- the single-band per-head RMSNorm + RoPE + paged store that
  * the fused_dual_qk_rms_norm_rope_ragged_paged page fuses twice (its first paragraph).
@@ -315,7 +318,7 @@ rope_status_t rope_split_store_paged_ragged_noalloc(
     const void *qkv, int64_t qkv_row_stride, int32_t total_tokens, int32_t n_q_heads,
     const uint32_t *input_row_offsets, int32_t batch, const rope_freqs_t *freqs,
     const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
-    uint32_t *err_word, rope_stream_t stream);
+    int32_t q_out_dtype, uint32_t *err_word, rope_stream_t stream);
 
 /* A static, human-readable name of a status code. */
 const char *rope_status_string(rope_status_t status);

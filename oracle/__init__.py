@@ -70,7 +70,7 @@ class _Band(ctypes.Structure):
                 ("k_col", _i64), ("v_col", _i64), ("n_q_heads", _i32),
                 ("cache", ctypes.POINTER(_Paged)), ("q_gamma", _c_void_p),
                 ("k_gamma", _c_void_p), ("epsilon", ctypes.c_double), ("q_out", _c_void_p),
-                ("q_out_row_stride", _i64), ("written", _c_void_p)]
+                ("q_out_row_stride", _i64), ("written", _c_void_p), ("q_out_dtype", _i32)]
 
 
 _lib = None
@@ -83,7 +83,7 @@ def _load():
         P = ctypes.POINTER
         lib.orc_rope_split_store_paged_ragged.argtypes = [
             _i32, _c_void_p, _i64, _i32, _i32, _c_void_p, _i32, P(_Rope), P(_Paged), _u32,
-            _c_void_p, _i64, _c_void_p]
+            _c_void_p, _i64, _i32, _c_void_p]
         lib.orc_fused_qk_rmsnorm_rope_paged.argtypes = [
             _i32, P(_Band), _c_void_p, _i32, _i32, P(_Rope), ctypes.c_double, _i32, _u32]
         lib.orc_fused_dual_qk_rmsnorm_rope_paged.argtypes = [
@@ -223,20 +223,20 @@ def _band(b: Band, keep: list) -> _Band:
     keep.append(pc)
     return _Band(_ptr(b.input), _row_stride(b.input), b.q_col, b.k_col, b.v_col, b.n_q_heads,
                  ctypes.pointer(pc), _ptr(b.q_gamma), _ptr(b.k_gamma), float(b.epsilon),
-                 _ptr(b.q_out), _row_stride(b.q_out), _ptr(b.written))
+                 _ptr(b.q_out), _row_stride(b.q_out), _ptr(b.written), -1)
 
 
 # ------------------------------------------------------------------------ operations --
 
 def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, rope: Rope,
                                   cache: PagedCache, layer_idx, q_out, written=None,
-                                  dtype="bf16") -> int:
+                                  dtype="bf16", q_out_dtype=None) -> int:
     offs = _as_u32(input_row_offsets)
     pc, rp = _paged(cache), _rope(rope)
     return _load().orc_rope_split_store_paged_ragged(
         DTYPES[dtype], _ptr(qkv), _row_stride(qkv), qkv.shape[0], n_q_heads, _ptr(offs),
         offs.shape[0] - 1, ctypes.byref(rp), ctypes.byref(pc), layer_idx, _ptr(q_out),
-        _row_stride(q_out), _ptr(written))
+        _row_stride(q_out), DTYPES[q_out_dtype] if q_out_dtype else -1, _ptr(written))
 
 
 def fused_qk_rmsnorm_rope_paged(band: Band, input_row_offsets, rope: Rope, weight_offset=0.0,

@@ -235,7 +235,9 @@ static uint32_t apply_band(int32_t dtype, orc_band *bd, const uint32_t *offs, in
       for (int32_t d = 0; d < D; ++d) y[d] = orc_decode(dtype, bd->input, in_row + bd->q_col + (int64_t)h * D + d);
       if (do_norm) rmsnorm_head(dtype, y, D, bd->q_gamma, eps, weight_offset, mbc);
       rope_head(y, D, rope, cs);
-      for (int32_t d = 0; d < D; ++d) orc_encode(dtype, bd->q_out, row * bd->q_out_row_stride + (int64_t)h * D + d, y[d]);
+      for (int32_t d = 0; d < D; ++d)
+        orc_encode(bd->q_out_dtype >= 0 ? bd->q_out_dtype : dtype, bd->q_out,
+                   row * bd->q_out_row_stride + (int64_t)h * D + d, y[d]);
     }
     for (int32_t h = 0; h < Hk; ++h) { /* K heads -> K cache (k_col < 0: K is the cache's) */
       for (int32_t d = 0; d < D; ++d)
@@ -271,15 +273,18 @@ uint32_t orc_rope_split_store_paged_ragged(int32_t dtype, const void *qkv, int64
                                            const uint32_t *input_row_offsets, int32_t batch,
                                            const orc_rope *rope, orc_paged_cache *kv,
                                            uint32_t layer_idx, void *q_out,
-                                           int64_t q_out_row_stride, uint8_t *written) {
+                                           int64_t q_out_row_stride, int32_t q_out_dtype,
+                                           uint8_t *written) {
   if (layer_idx >= (uint32_t)kv->num_layers || batch > kv->n_seqs ||
       !rope_geometry_ok(rope, kv->head_dim) || kv->v == NULL)
     return ORC_ERR_ARGS;
   uint32_t e = check_row_offsets(input_row_offsets, batch, total_tokens);
   if (e) return e;
   int64_t D = kv->head_dim;
+  /* [P2] q_out_dtype: the element type of the Q output (the input's by default) */
   orc_band bd = {qkv, qkv_row_stride, 0, n_q_heads * D, (n_q_heads + kv->n_kv_heads) * D,
-                 n_q_heads, kv, NULL, NULL, 0.0, q_out, q_out_row_stride, written};
+                 n_q_heads, kv, NULL, NULL, 0.0, q_out, q_out_row_stride, written,
+                 q_out_dtype};
   return apply_band(dtype, &bd, input_row_offsets, batch, total_tokens, rope, 0, 0.0, 1,
                     layer_idx);
 }

@@ -91,6 +91,7 @@ typedef struct {
   void *q_out;
   int64_t q_out_row_stride;
   uint8_t *written; /* optional [num_pages*page_size]: set to 1 for each (page, slot) stored */
+  int32_t q_out_dtype; /* element type of q_out; < 0: the input's */
 } orc_band;
 
 uint32_t orc_rope_split_store_paged_ragged(int32_t dtype, const void *qkv, int64_t qkv_row_stride,
@@ -98,7 +99,8 @@ uint32_t orc_rope_split_store_paged_ragged(int32_t dtype, const void *qkv, int64
                                            const uint32_t *input_row_offsets, int32_t batch,
                                            const orc_rope *rope, orc_paged_cache *kv,
                                            uint32_t layer_idx, void *q_out,
-                                           int64_t q_out_row_stride, uint8_t *written);
+                                           int64_t q_out_row_stride, int32_t q_out_dtype,
+                                           uint8_t *written);
 
 uint32_t orc_fused_qk_rmsnorm_rope_paged(int32_t dtype, orc_band *band,
                                          const uint32_t *input_row_offsets, int32_t batch,

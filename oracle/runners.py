@@ -60,8 +60,11 @@ def oracle_ragged_store(w: "W.RaggedStore", dtype: str = "bf16",
     cache = oracle_paged(w.cache, store)
     rope = oracle_rope(w.rope)
     if w.q_gamma is None:
+        q_dtype = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[
+            w.q_out.dtype]
         err = oracle.rope_split_store_paged_ragged(qkv, w.n_q_heads, bits(w.offsets), rope,
-                                                   cache, w.layer_idx, q_out, written, dtype)
+                                                   cache, w.layer_idx, q_out, written, dtype,
+                                                   q_dtype)
     else:
         D = w.cache.head_dim
         Hq, Hk = w.n_q_heads, w.cache.n_kv_heads

@@ -89,8 +89,8 @@ class c_norm_band(ctypes.Structure):
 
 _P = ctypes.POINTER
 _lib.rope_split_store_paged_ragged.argtypes = [
-    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp,
-    _vp, _vp]
+    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _i32,
+    _vp, _vp, _vp]
 _lib.fused_qk_rmsnorm_rope_paged.argtypes = [
     _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _vp, _vp, _f32, _f32,
     _i32, _u32, _vp, _i64, _vp, _vp, _vp]
@@ -102,8 +102,8 @@ _lib.qk_rope_bshd_continuous.argtypes = [
 _lib.kv_cache_radd.argtypes = [
     _vp, _i64, _i32, _P(c_paged_cache), _vp, _i32, _u32, _u32, _vp, _vp, _vp]
 _lib.rope_split_store_paged_ragged_noalloc.argtypes = [
-    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _vp,
-    _vp]
+    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _i32,
+    _vp, _vp]
 _lib.matmul_fused_partial_rmsnorm.argtypes = [
     _vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _f32, _vp, _i32, _vp, _i32, _vp, _vp, _i64,
     _vp]
@@ -283,8 +283,8 @@ def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, freqs: Freq
     _check(_lib.rope_split_store_paged_ragged(
         qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
-        _row_stride(q_out), _ptr(err_word), _sched(sched), _stream(stream)),
-        "rope_split_store_paged_ragged")
+        _row_stride(q_out), _DTYPE_CODE[q_out.dtype], _ptr(err_word), _sched(sched),
+        _stream(stream)), "rope_split_store_paged_ragged")
 
 
 def rope_split_store_paged_ragged_noalloc(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
@@ -298,7 +298,7 @@ def rope_split_store_paged_ragged_noalloc(qkv, n_q_heads, input_row_offsets, fre
     _check(_lib.rope_split_store_paged_ragged_noalloc(
         qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
-        _row_stride(q_out), _ptr(err_word), _stream(stream)),
+        _row_stride(q_out), _DTYPE_CODE[q_out.dtype], _ptr(err_word), _stream(stream)),
         "rope_split_store_paged_ragged_noalloc")
 
 

@@ -52,7 +52,39 @@ struct BandDev {
   int32_t seg_bytes[3], seg_dst[3];
   int32_t kv_contig;  // a slot's heads are adjacent in the cache (one store per plane)
   int32_t k_inplace;  // K heads come from the token's cache slot, not from the input
+  // Q output in another element type: the consumers write the rotated Q rows, converted,
+  // to a stage region at qo_off, from where the storer copies them
+  int32_t q_conv, q_dtype, q_eb, qo_off;
 };
+
+// N float values written to shared memory as N elements of type qd (0 bf16, 1 f16, 2 f32),
+// rounded to nearest even
+template <int N>
+__device__ __forceinline__ void st_shared_elems(unsigned char *p, const float (&x)[N], int qd) {
+  if (qd == 2) {
+#pragma unroll
+    for (int k = 0; k < N; k += 4)
+      st_shared_v4(p + k * 4, make_uint4(__float_as_uint(x[k]), __float_as_uint(x[k + 1]),
+                                         __float_as_uint(x[k + 2]), __float_as_uint(x[k + 3])));
+    return;
+  }
+  uint32_t w[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    if (qd == 0) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t *>(&h);
+    } else {
+      __half2 h = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t *>(&h);
+    }
+  }
+  if constexpr (N == 8) {
+    st_shared_v4(p, make_uint4(w[0], w[1], w[2], w[3]));
+  } else {
+    st_shared_v2(p, w[0], w[1]);
+  }
+}
 
 struct BandedParams {
   BandDev band[2];
@@ -211,7 +243,8 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
 template <int CW>
 __host__ __device__ constexpr int pipe_min_ctas() { return CW <= 4 ? ROPE_LIGHT_MIN_CTAS : 2; }
 
-template <typename T, int D, bool NORM, int CW, int LAG>
+// QCONV: built with the Q-output conversion (only the store without RMSNorm uses it)
+template <typename T, int D, bool NORM, int CW, int LAG, bool QCONV>
 __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     banded_store_kernel(const __grid_constant__ BandedParams p) {
   constexpr int kConsumerWarps = CW;
@@ -437,10 +470,16 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
           const BandDev &bd = k ? p.band[1] : p.band[0];
           const unsigned char *blk = st + bd.smem_off;
           const uint32_t qb = (uint32_t)(bd.n_q * D * EB), kb = (uint32_t)(bd.n_kv * D * EB);
-          if (qb)
-            bulk_s2g(reinterpret_cast<unsigned char *>(bd.q_out) +
-                         (int64_t)tok * bd.q_out_stride * EB,
-                     blk, qb);
+          if (qb) {
+            if (bd.q_conv)  // the converted rows
+              bulk_s2g(reinterpret_cast<unsigned char *>(bd.q_out) +
+                           (int64_t)tok * bd.q_out_stride * bd.q_eb,
+                       st + bd.qo_off, (uint32_t)(bd.n_q * D * bd.q_eb));
+            else
+              bulk_s2g(reinterpret_cast<unsigned char *>(bd.q_out) +
+                           (int64_t)tok * bd.q_out_stride * EB,
+                       blk, qb);
+          }
           const int64_t base = meta[s].kv_base[k];
           for (int plane = 0; plane < (bd.n_v ? 2 : 1); ++plane) {
             unsigned char *dst = reinterpret_cast<unsigned char *>(plane ? bd.cache.v : bd.cache.k) +
@@ -544,11 +583,13 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
 #pragma unroll 1
       for (int u = 0; u < n_items; ++u) {
         const uint32_t w = item[u * kConsumers];
-        if (!busy || !(w & kItemAct)) continue;
+        if (!(w & kItemAct)) continue;
         const int band = (w >> kItemBandShift) & 1;
         if (!(band ? ok1 : ok0)) continue;
         const int kind = (w >> kItemKindShift) & 1;
         const BandDev &bd = band ? p.band[1] : p.band[0];
+        const bool conv = QCONV && kind == 0 && bd.q_conv;  // every lane writes its Q
+        if (!busy && !conv) continue;
         if ((rot_a || rot_b) && f_band != band) {  // this token's table row for the band
           f_band = band;
           const unsigned char *F = st + bd.f_off;
@@ -656,8 +697,15 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
             xb[e] = yb.x; xb[e + 1] = yb.y;
           }
         }
-        if (NORM || rot_a) st_shared_v4(row + ca * EB, VT::narrow(xa));
-        if (NORM || rot_b) st_shared_v4(row + cb * EB, VT::narrow(xb));
+        if (conv) {
+          unsigned char *qrow = st + bd.qo_off +
+                                (size_t)(((w & kItemOffMask) - bd.smem_off) / EB) * bd.q_eb;
+          st_shared_elems<N>(qrow + ca * bd.q_eb, xa, bd.q_dtype);
+          st_shared_elems<N>(qrow + cb * bd.q_eb, xb, bd.q_dtype);
+        } else {
+          if (NORM || rot_a) st_shared_v4(row + ca * EB, VT::narrow(xa));
+          if (NORM || rot_b) st_shared_v4(row + cb * EB, VT::narrow(xb));
+        }
       }
       fence_proxy_async_smem();  // the storer's bulk copies read what was written here
       __syncwarp();

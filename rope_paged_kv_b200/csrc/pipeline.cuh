@@ -137,6 +137,11 @@ __device__ __forceinline__ void st_shared_v4(void *p, uint4 v) {
                : "memory");
 }
 
+__device__ __forceinline__ void st_shared_v2(void *p, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(smem_addr(p)), "r"(a), "r"(b)
+               : "memory");
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"

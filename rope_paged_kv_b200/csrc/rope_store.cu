@@ -52,7 +52,8 @@ static int passes(const BandedParams &p, int D, int cw) {
 }
 
 static ShapeId pick_shape(const BandedParams &p, int D, bool norm) {
-  if (!norm && p.work_total <= 64) return kLight;
+  // the light shape is the one built with the Q-output conversion
+  if (!norm && (p.work_total <= 64 || p.band[0].q_conv)) return kLight;
   return passes(p, D, kMidShape.cw) <= passes(p, D, kHeavyShape.cw) ? kMid : kHeavy;
 }
 
@@ -208,7 +209,7 @@ static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride
                                int64_t k_col, int64_t v_col, int32_t n_q,
                                const rope_paged_cache_t *kv, const void *qg, const void *kg,
                                float eps, void *q_out, int64_t q_out_stride, int dtype,
-                               uint32_t layer, bool norm) {
+                               uint32_t layer, bool norm, int q_dtype = -1) {
   if (input == nullptr || q_out == nullptr || n_q < 0 || in_stride < 0 || q_out_stride < 0 ||
       q_col < 0)
     return ROPE_ERR_INVALID_ARG;
@@ -218,12 +219,15 @@ static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride
   if (s != ROPE_OK) return s;
   const int64_t D = kv->head_dim, Hk = kv->n_kv_heads;
   const int eb = elem_bytes(dtype);
+  if (q_dtype < 0) q_dtype = dtype;
+  const int qeb = elem_bytes(q_dtype);
+  if (qeb == 0 || (norm && q_dtype != dtype)) return ROPE_ERR_UNSUPPORTED;
   const int64_t nv = v_col >= 0 ? Hk : 0;
   if (in_stride < q_col + n_q * D || (!k_inplace && in_stride < k_col + Hk * D) ||
       (v_col >= 0 && in_stride < v_col + Hk * D) || q_out_stride < n_q * D)
     return ROPE_ERR_INVALID_ARG;
   if (!aligned16(input) || !aligned16(q_out) || !stride16(in_stride, eb) ||
-      !stride16(q_out_stride, eb) || !stride16(q_col, eb) ||
+      !stride16(q_out_stride, qeb) || !stride16(q_col, eb) ||
       (!k_inplace && !stride16(k_col, eb)) || (v_col >= 0 && !stride16(v_col, eb)))
     return ROPE_ERR_UNSUPPORTED;
   bd->input = input;
@@ -241,6 +245,9 @@ static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride
   bd->eps = eps;
   bd->kv_contig = kv->head_stride == D ? 1 : 0;
   bd->k_inplace = k_inplace ? 1 : 0;
+  bd->q_conv = q_dtype != dtype ? 1 : 0;
+  bd->q_dtype = q_dtype == ROPE_DTYPE_F32 ? 2 : q_dtype == ROPE_DTYPE_F16 ? 1 : 0;
+  bd->q_eb = qeb;
   // staging segments: Q, K, V blocks (merged when adjacent in the input row); an in-place
   // K block keeps its place in the stage but is loaded from the cache
   const int64_t cols[3] = {q_col, k_col, v_col};
@@ -296,6 +303,11 @@ static size_t layout_banded(BandedParams &p, int D, bool norm, const BandedShape
     p.band[k].f_off = (int32_t)off;
     off = round_up(off + p.f_row_bytes, 16);
   }
+  for (int k = 0; k < p.n_bands; ++k) {  // converted Q rows
+    BandDev &bd = p.band[k];
+    bd.qo_off = (int32_t)off;
+    if (bd.q_conv) off = round_up(off + (int64_t)bd.n_q * D * bd.q_eb, 16);
+  }
   p.stage_bytes = (int32_t)round_up(off, 128);
   int S = (int)(kStageTarget / p.stage_bytes);
   // the storer holds up to kStoreLag + 1 stages; keep at least two for loading / compute
@@ -318,10 +330,10 @@ static size_t layout_banded(BandedParams &p, int D, bool norm, const BandedShape
   return (size_t)round_up(total, 128);
 }
 
-template <typename T, int D, bool NORM, int CW, int LAG>
+template <typename T, int D, bool NORM, int CW, int LAG, bool QCONV = false>
 static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStream_t st) {
   static ShapeCache cache;
-  auto kern = banded_store_kernel<T, D, NORM, CW, LAG>;
+  auto kern = banded_store_kernel<T, D, NORM, CW, LAG, QCONV>;
   const int occ = resident_ctas(kern, pipe_threads<CW>(), smem, cache);
   if (occ <= 0) return ROPE_ERR_UNSUPPORTED;  // the stage ring does not fit
   const int64_t slots = (int64_t)sm_count() * occ;
@@ -332,8 +344,13 @@ static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStr
 template <typename T, int D, bool NORM>
 static rope_status_t launch_banded_s(ShapeId id, const BandedParams &p, size_t smem,
                                      cudaStream_t st) {
-  if (id == kLight)
+  if (id == kLight) {
+    if constexpr (!NORM) {
+      if (p.band[0].q_conv)  // Q written in another element type
+        return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag, true>(p, smem, st);
+    }
     return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
+  }
   if (id == kMid) return launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag>(p, smem, st);
   return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag>(p, smem, st);
 }
@@ -512,8 +529,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
                                             const rope_freqs_t *freqs,
                                             const rope_paged_cache_t *kv, uint32_t layer_idx,
                                             void *q_out, int64_t q_out_row_stride,
-                                            uint32_t *err_word, uint32_t *sched,
-                                            rope_stream_t stream) {
+                                            int32_t q_out_dtype, uint32_t *err_word,
+                                            uint32_t *sched, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
   if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
   const int dtype = kv->dtype, D = kv->head_dim;
@@ -525,7 +542,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
   if (s != ROPE_OK) return s;
   const int64_t Hq = n_q_heads, Hk = kv->n_kv_heads;
   s = fill_band(&p.band[0], qkv, qkv_row_stride, 0, Hq * D, (Hq + Hk) * D, n_q_heads, kv,
-                nullptr, nullptr, 0.f, q_out, q_out_row_stride, dtype, layer_idx, false);
+                nullptr, nullptr, 0.f, q_out, q_out_row_stride, dtype, layer_idx, false,
+                q_out_dtype);
   if (s != ROPE_OK) return s;
   p.n_bands = 1;
   p.work0 = p.work_total = (int32_t)(Hq + Hk);
@@ -719,7 +737,7 @@ rope_status_t rope_split_store_paged_ragged_noalloc(
     const void *qkv, int64_t qkv_row_stride, int32_t total_tokens, int32_t n_q_heads,
     const uint32_t *input_row_offsets, int32_t batch, const rope_freqs_t *freqs,
     const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
-    uint32_t *err_word, rope_stream_t stream) {
+    int32_t q_out_dtype, uint32_t *err_word, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
   uint32_t *scratch = noalloc_scratch();
   if (scratch == nullptr) return ROPE_ERR_CUDA;
@@ -729,7 +747,8 @@ rope_status_t rope_split_store_paged_ragged_noalloc(
     return ROPE_ERR_CUDA;
   return rope_split_store_paged_ragged(qkv, qkv_row_stride, total_tokens, n_q_heads,
                                        input_row_offsets, batch, freqs, kv, layer_idx, q_out,
-                                       q_out_row_stride, err_word, scratch, stream);
+                                       q_out_row_stride, q_out_dtype, err_word, scratch,
+                                       stream);
 }
 
 rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight,

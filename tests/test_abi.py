@@ -75,7 +75,8 @@ def test_host_argument_checks_need_no_gpu(rs):
     f = rs.c_freqs(fake, 2, 64, 64, 1, -1)
     kv = rs.c_paged_cache(fake, fake, 0, 2, 64, 16, 8, 2, 4096, 2048, 128, 64, fake, 4, 4,
                           fake, 2)
-    call = lib.rope_split_store_paged_ragged
+    def call(*a):  # the store with q_out in the cache's element type
+        return lib.rope_split_store_paged_ragged(*a[:11], -1, *a[11:])
     # NULL descriptors / pointers
     assert call(fake, 512, 8, 4, fake, 2, None, ctypes.byref(kv), 1, fake, 256, None, None,
                 None) == rs.ERR_INVALID_ARG
@@ -109,10 +110,14 @@ def test_host_argument_checks_need_no_gpu(rs):
     # empty work: OK without a launch
     assert call(fake, 512, 0, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
                 None, None, None) == rs.OK
-    # multiply_before_cast = 0 is not built
+    # the norm op needs both gammas (checked before any launch)
     assert lib.fused_qk_rmsnorm_rope_paged(fake, 512, 8, 4, fake, 2, ctypes.byref(f),
-                                           ctypes.byref(kv), fake, fake, 1e-6, 0.0, 0, 1, fake,
-                                           256, None, None, None) == rs.ERR_UNSUPPORTED
+                                           ctypes.byref(kv), None, fake, 1e-6, 0.0, 0, 1, fake,
+                                           256, None, None, None) == rs.ERR_INVALID_ARG
+    # a q_out element type that does not exist
+    assert lib.rope_split_store_paged_ragged(fake, 512, 8, 4, fake, 2, ctypes.byref(f),
+                                             ctypes.byref(kv), 1, fake, 256, 7, None, None,
+                                             None) == rs.ERR_UNSUPPORTED
     # dual band: geometry must agree across bands
     kv128 = rs.c_paged_cache(fake, None, 0, 1, 128, 16, 8, 2, 4096, 2048, 128, 128, fake, 4,
                              4, fake, 2)

@@ -62,3 +62,26 @@ def test_multiply_after_cast_ragged(G, head_dim, dtype):
 def test_multiply_after_cast_dual_in_place(G):
     w = band_case(44, k_in_place=True, x_std=2.0)
     _check_dual(G, w, G.run_dual(w, multiply_before_cast=False), multiply_before_cast=False)
+
+
+@pytest.mark.parametrize("dtype,q_dtype,head_dim", [
+    ("bf16", "f32", 128), ("bf16", "f16", 128), ("f16", "bf16", 64), ("f32", "bf16", 64),
+    ("f32", "f16", 128), ("bf16", "bf16", 128)])
+@pytest.mark.parametrize("interleaved", [True, False])
+def test_q_out_element_type(G, dtype, q_dtype, head_dim, interleaved):
+    # rope_split_store_paged_ragged's q_out_dtype: Q rounded once into its own type;
+    # partial rope so that unrotated columns are converted too
+    w = W.ragged_store(45, lengths=[300, 2, 257], cache_lengths=[0, 5, 64], n_q_heads=8,
+                       n_kv_heads=2, head_dim=head_dim, page_size=32, rope_dim=head_dim // 2,
+                       theta=1e4, interleaved=interleaved, max_seq_len=1024, dtype=dtype,
+                       q_out_dtype=q_dtype)
+    check_ragged(G, w, G.run_ragged(w))
+
+
+def test_q_out_element_type_many_heads(G):
+    # more head rows than the light shape's usual share: the call still takes the shape
+    # built with the conversion
+    w = W.ragged_store(46, lengths=[130, 70], cache_lengths=[0, 9], n_q_heads=64,
+                       n_kv_heads=8, head_dim=128, page_size=64, rope_dim=128, theta=5e5,
+                       interleaved=False, max_seq_len=512, q_out_dtype="f32")
+    check_ragged(G, w, G.run_ragged(w))

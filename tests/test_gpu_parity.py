@@ -58,8 +58,9 @@ def check_ragged(G, w, s, exact_norm_cols=False, multiply_before_cast=True):
             w.cache.cache_lengths.tolist(), w.lengths, w.layer_idx)
     q = H.bits(s.q_out).reshape(T, Hq, D)
     qo = r.q_out.reshape(T, Hq, D)
+    qd = {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[w.q_out.dtype]
     H.assert_bits_equal(q[..., ~fpc], qo[..., ~fpc], "q_out pass-through columns")
-    H.assert_close_bf16(q[..., fpc], qo[..., fpc], "q_out", dtype=w.cache.dtype, extra=eq)
+    H.assert_close_bf16(q[..., fpc], qo[..., fpc], "q_out", dtype=qd, extra=eq)
     H.compare_paged_cache(w.cache, H.bits(s.storage), r.storage, r.written, w.layer_idx, fpc,
                           "cache", k_extra=ek)
     return r

@@ -675,3 +675,44 @@ def test_gemv_weight_offset_is_not_consumed_and_partitions_agree():
                     W.random_bits(W.generator(1), 30, "bf16"))
     z = H.oracle_gemv(w0, "bf16")
     assert np.array_equal(z.unnormed[10:], a.unnormed)
+
+
+# ------------------------------------------------------- Q output in another element type --
+
+def test_q_out_f32_at_position_zero_is_the_input_widened():
+    # rope_split_store_paged_ragged, Parameters: q_out_dtype.  At position 0 the rotation is
+    # the identity, so a float32 q_out holds the bf16 input exactly
+    w = W.ragged_store(130, lengths=[1, 1, 1], cache_lengths=[0, 0, 0], n_q_heads=4,
+                       n_kv_heads=2, head_dim=64, page_size=8, rope_dim=64, theta=1e4,
+                       interleaved=True, max_seq_len=16, q_out_dtype="f32")
+    r = H.oracle_ragged_store(w, "bf16")
+    assert r.err == 0
+    want = w.qkv[:, :4 * 64].float().numpy()
+    np.testing.assert_array_equal(r.q_out.view(np.float32), want)
+
+
+@pytest.mark.parametrize("q_dtype", ["f32", "f16"])
+def test_q_out_in_another_type_is_the_same_value_rounded_once(q_dtype):
+    # the same rotated value rounded once into each type: the bf16 output lies within half a
+    # bf16 spacing of the wider one, and the f32 output is the complex product of the pages'
+    # interleaved layout, rounded once
+    kw = dict(lengths=[5, 9], cache_lengths=[3, 40], n_q_heads=2, n_kv_heads=1, head_dim=64,
+              page_size=16, rope_dim=64, theta=1e4, interleaved=True, max_seq_len=64)
+    a = H.oracle_ragged_store(W.ragged_store(131, **kw), "bf16")
+    wq = W.ragged_store(131, q_out_dtype=q_dtype, **kw)
+    b = H.oracle_ragged_store(wq, "bf16")
+    assert a.err == b.err == 0
+    qa = H.values(a.q_out, "bf16")
+    qb = H.values(b.q_out, q_dtype)
+    assert bool(np.all(np.abs(qa - qb) <= 0.5 * H.bf16_ulp(qa) + 0.5 * H.ulp_of(qb, q_dtype)))
+    assert np.array_equal(a.storage, b.storage)
+    if q_dtype == "f32":
+        T = wq.total_tokens
+        x = wq.qkv[:, :2 * 64].double().numpy().reshape(T, 2, 32, 2)
+        z = x[..., 0] + 1j * x[..., 1]
+        pos = np.concatenate([np.arange(3, 8), np.arange(40, 49)])
+        f = wq.rope.table.double().numpy()[pos].reshape(T, 1, 32, 2)
+        y = z * (f[..., 0] + 1j * f[..., 1])
+        got = qb.reshape(T, 2, 32, 2)
+        sp = np.spacing(np.abs(np.stack([y.real, y.imag], -1)).astype(np.float32))
+        assert bool(np.all(np.abs(got - np.stack([y.real, y.imag], -1)) <= 0.5 * sp * (1 + 1e-9)))

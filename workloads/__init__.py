@@ -253,7 +253,8 @@ def ragged_store(seed: int, *, lengths: List[int], cache_lengths: List[int], n_q
                  x_std: float = 1.0, norm: bool = False, epsilon: float = 1e-6,
                  weight_offset: float = 0.0, num_layers: int = 2, layer_idx: int = 1,
                  width: Optional[int] = None, rope_col_offset: int = -1,
-                 dtype: str = "bf16", row_pad: int = 0, name: str = "") -> RaggedStore:
+                 dtype: str = "bf16", row_pad: int = 0, q_out_dtype: Optional[str] = None,
+                 name: str = "") -> RaggedStore:
     gen = generator(seed)
     T = sum(lengths)
     D = head_dim
@@ -266,7 +267,7 @@ def ragged_store(seed: int, *, lengths: List[int], cache_lengths: List[int], n_q
                         dtype=dtype)
     rope = RopeSpec(freqs_cis(max_seq_len, rope_dim, theta, freq_dtype), freq_dtype,
                     interleaved, rope_col_offset)
-    q_out = random_bits(gen, T * n_q_heads * D, dtype).view(T, n_q_heads * D)
+    q_out = random_bits(gen, T * n_q_heads * D, q_out_dtype or dtype).view(T, n_q_heads * D)
     w = ragged_store_gammas(gen, D, dtype) if norm else (None, None)
     return RaggedStore(qkv, row_offsets(lengths), n_q_heads, cache, rope, layer_idx, q_out,
                        list(lengths), w[0], w[1], epsilon, weight_offset, name)
