@@ -352,6 +352,10 @@ static rope_status_t launch_banded_s(ShapeId id, const BandedParams &p, size_t s
     return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
   }
   if (id == kMid) return launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag>(p, smem, st);
+  if constexpr (!NORM) {
+    if (p.band[0].q_conv)  // stages too large for the light ring
+      return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag, true>(p, smem, st);
+  }
   return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag>(p, smem, st);
 }
 
@@ -368,8 +372,14 @@ static rope_status_t launch_banded_d(int D, ShapeId id, const BandedParams &p, s
 static rope_status_t launch_banded(int dtype, int D, bool norm, BandedParams &p,
                                    cudaStream_t st) {
   p.elem_bytes = elem_bytes(dtype);
-  const ShapeId id = pick_shape(p, D, norm);
-  const size_t smem = layout_banded(p, D, norm, shape_of(id));
+  ShapeId id = pick_shape(p, D, norm);
+  const BandedParams unplaced = p;  // layout_banded places the stage offsets in p
+  size_t smem = layout_banded(p, D, norm, shape_of(id));
+  if (smem > 227 * 1024 && id == kLight) {  // stages too large for its ring of >= 5
+    p = unplaced;
+    id = kHeavy;
+    smem = layout_banded(p, D, norm, kHeavyShape);
+  }
   if (smem > 227 * 1024) return ROPE_ERR_UNSUPPORTED;
   if (dtype == ROPE_DTYPE_BF16)
     return norm ? launch_banded_d<__nv_bfloat16, true>(D, id, p, smem, st)
