@@ -19,6 +19,9 @@ Parity status of the functions (what pins each one is stated in the test-suite):
   multiply, and only its reduction to the plain op at unit gamma is checked).
   The choice of rotated columns under partial RoPE is a reading of an open point; it is
   pinned only against the reading it implements.
+  FP8 (E4M3) caches: the element codec is pinned against torch's float8_e4m3fn; the format
+  around it (one float32 scale per K / V plane, code = e4m3(value / scale), saturating) is
+  parity unpinned: the pages name a scale type and a quantisation granularity only.
 """
 from __future__ import annotations
 
@@ -30,7 +33,7 @@ import numpy as np
 
 from . import build as _build
 
-DTYPES = {"bf16": 0, "f16": 1, "f32": 2}
+DTYPES = {"bf16": 0, "f16": 1, "f32": 2, "fp8": 3}  # fp8: OCP E4M3 (cache elements only)
 ERR_ROW_OFFSETS = 0x1
 ERR_POSITION = 0x2
 ERR_PAGE_INDEX = 0x4
@@ -48,7 +51,8 @@ class _Paged(ctypes.Structure):
                 ("num_pages", _i32), ("num_layers", _i32),
                 ("page_stride", _i64), ("layer_stride", _i64), ("slot_stride", _i64),
                 ("head_stride", _i64), ("page_table", _c_void_p), ("page_table_stride", _i64),
-                ("max_pages_per_seq", _i32), ("cache_lengths", _c_void_p), ("n_seqs", _i32)]
+                ("max_pages_per_seq", _i32), ("cache_lengths", _c_void_p), ("n_seqs", _i32),
+                ("k_scale", _c_void_p), ("v_scale", _c_void_p)]
 
 
 class _Cont(ctypes.Structure):
@@ -134,6 +138,8 @@ class PagedCache:
     page_table: np.ndarray      # uint32 [n_seqs, width]
     max_pages_per_seq: int
     cache_lengths: np.ndarray   # uint32 [n_seqs]
+    k_scale: Optional[np.ndarray] = None  # float32 [1] each, for an fp8 cache
+    v_scale: Optional[np.ndarray] = None
 
 
 @dataclass
@@ -208,7 +214,7 @@ def _paged(c: PagedCache) -> _Paged:
                   DTYPES[c.dtype], c.n_kv_heads, c.head_dim, c.page_size, c.num_pages,
                   c.num_layers, c.page_stride, c.layer_stride, c.slot_stride, c.head_stride,
                   _ptr(pt), pt.shape[1], c.max_pages_per_seq, _ptr(_as_u32(c.cache_lengths)),
-                  pt.shape[0])
+                  pt.shape[0], _ptr(c.k_scale), _ptr(c.v_scale))
 
 
 def _rope(r: Rope) -> _Rope:

@@ -105,9 +105,40 @@ static uint16_t double_to_f16_bits(double v) {
   return sign | (uint16_t)(ex << 10) | m;
 }
 
+/* OCP 8-bit E4M3 ("fn": no infinities): sign, 4 exponent bits biased by 7, 3 fraction bits;
+ * exponent 15 with fraction 7 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448. */
+static double e4m3_bits_to_double(uint8_t h) {
+  int neg = h >> 7, e = (h >> 3) & 15, m = h & 7;
+  double v;
+  if (e == 15 && m == 7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)m, -9); /* subnormal: m * 2^-9 */
+  else
+    v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+  return neg ? -v : v;
+}
+
+/* nearest E4M3 value, ties to even, saturating: magnitudes past 448 (and infinities)
+ * become 448 */
+static uint8_t double_to_e4m3_bits(double v) {
+  if (isnan(v)) return 0x7F;
+  uint8_t sign = signbit(v) ? 0x80 : 0;
+  double a = fabs(v);
+  if (a == 0.0) return sign;
+  double r = isinf(a) ? 448.0 : round_to_grid(a, 3, -6);
+  if (r > 448.0) r = 448.0;
+  if (r < ldexp(1.0, -6)) return sign | (uint8_t)ldexp(r, 9); /* subnormal */
+  int e;
+  double f = frexp(r, &e); /* r = (1 + m/8) * 2^(e-1) */
+  uint8_t m = (uint8_t)(ldexp(f, 4) - 8.0);
+  return sign | (uint8_t)((e - 1 + 7) << 3) | m;
+}
+
 double orc_decode(int32_t dtype, const void *base, int64_t i) {
   if (dtype == ORC_BF16) return bf16_bits_to_double(((const uint16_t *)base)[i]);
   if (dtype == ORC_F16) return f16_bits_to_double(((const uint16_t *)base)[i]);
+  if (dtype == ORC_FP8_E4M3) return e4m3_bits_to_double(((const uint8_t *)base)[i]);
   return (double)((const float *)base)[i];
 }
 
@@ -116,8 +147,24 @@ void orc_encode(int32_t dtype, void *base, int64_t i, double v) {
     ((uint16_t *)base)[i] = double_to_bf16_bits(v);
   else if (dtype == ORC_F16)
     ((uint16_t *)base)[i] = double_to_f16_bits(v);
+  else if (dtype == ORC_FP8_E4M3)
+    ((uint8_t *)base)[i] = double_to_e4m3_bits(v);
   else
     ((float *)base)[i] = (float)v; /* C conversion: round to nearest even */
+}
+
+/* A cache element: an FP8 cache holds code = e4m3(value / scale) with one float32 scale per
+ * plane (the scale_dtype_ / quantization_granularity_ of the pages' cache collections, read
+ * as per-tensor scales); other caches hold the value. */
+static double cache_scale(const orc_paged_cache *c, int plane) {
+  if (c->dtype != ORC_FP8_E4M3) return 1.0;
+  return (double)*(plane ? c->v_scale : c->k_scale);
+}
+static double cache_get(const orc_paged_cache *c, int plane, int64_t i) {
+  return orc_decode(c->dtype, plane ? c->v : c->k, i) * cache_scale(c, plane);
+}
+static void cache_put(const orc_paged_cache *c, int plane, int64_t i, double v) {
+  orc_encode(c->dtype, plane ? c->v : c->k, i, v / cache_scale(c, plane));
 }
 
 /* the value v takes once stored in `dtype` */
@@ -243,16 +290,16 @@ static uint32_t apply_band(int32_t dtype, orc_band *bd, const uint32_t *offs, in
       for (int32_t d = 0; d < D; ++d)
         y[d] = bd->k_col >= 0
                    ? orc_decode(dtype, bd->input, in_row + bd->k_col + (int64_t)h * D + d)
-                   : orc_decode(c->dtype, c->k, base + h * c->head_stride + d);
+                   : cache_get(c, 0, base + h * c->head_stride + d);
       if (do_norm) rmsnorm_head(dtype, y, D, bd->k_gamma, eps, weight_offset, mbc);
       rope_head(y, D, rope, cs);
-      for (int32_t d = 0; d < D; ++d) orc_encode(c->dtype, c->k, base + h * c->head_stride + d, y[d]);
+      for (int32_t d = 0; d < D; ++d) cache_put(c, 0, base + h * c->head_stride + d, y[d]);
     }
     if (bd->v_col >= 0) /* V heads -> V cache, unchanged */
       for (int32_t h = 0; h < Hk; ++h)
         for (int32_t d = 0; d < D; ++d)
-          orc_encode(c->dtype, c->v, base + h * c->head_stride + d,
-                     orc_decode(dtype, bd->input, in_row + bd->v_col + (int64_t)h * D + d));
+          cache_put(c, 1, base + h * c->head_stride + d,
+                    orc_decode(dtype, bd->input, in_row + bd->v_col + (int64_t)h * D + d));
     if (bd->written) bd->written[flat] = 1;
   }
   free(y);
@@ -412,8 +459,8 @@ uint32_t orc_kv_cache_radd(int32_t dtype, const void *a, int64_t a_row_stride,
         int64_t ce = base + h * kv->head_stride + d;
         double ak = orc_decode(dtype, a, row * a_row_stride + h * D + d);
         double av = orc_decode(dtype, a, row * a_row_stride + hidden + h * D + d);
-        orc_encode(kv->dtype, kv->k, ce, orc_decode(kv->dtype, kv->k, ce) + ak);
-        orc_encode(kv->dtype, kv->v, ce, orc_decode(kv->dtype, kv->v, ce) + av);
+        cache_put(kv, 0, ce, cache_get(kv, 0, ce) + ak);
+        cache_put(kv, 1, ce, cache_get(kv, 1, ce) + av);
       }
     if (written) written[flat] = 1;
   }

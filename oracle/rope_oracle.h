@@ -31,7 +31,7 @@ extern "C" {
 #endif
 
 /* element type codes */
-enum { ORC_BF16 = 0, ORC_F16 = 1, ORC_F32 = 2 };
+enum { ORC_BF16 = 0, ORC_F16 = 1, ORC_F32 = 2, ORC_FP8_E4M3 = 3 };
 
 /* data-dependent error bits (returned; same meaning as the device error word) */
 #define ORC_ERR_ROW_OFFSETS 0x1u /* input_row_offsets is not a partition of [0, T) */
@@ -54,6 +54,10 @@ typedef struct {
   int32_t max_pages_per_seq;
   const uint32_t *cache_lengths; /* [n_seqs] tokens already cached per sequence */
   int32_t n_seqs;
+  /* FP8 (ORC_FP8_E4M3) caches: one float32 scale per plane; an element holds
+   * e4m3(value / scale), rounded to nearest even and saturated at +-448.  Parity unpinned:
+   * the pages name a scale type and a quantisation granularity without defining them. */
+  const float *k_scale, *v_scale;
 } orc_paged_cache;
 
 /* A continuous-batching K/V cache: element (slot, layer, pos, head, d) of the K plane at

@@ -13,8 +13,10 @@ import oracle
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
-    """A host copy of a tensor's raw element bits (uint16 for 16-bit types)."""
+    """A host copy of a tensor's raw element bits (uint16 for 16-bit types, uint8 for fp8)."""
     t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy().copy()
     if t.dtype in (torch.bfloat16, torch.float16):
         return t.view(torch.int16).numpy().view(np.uint16).copy()
     if t.dtype == torch.float32:
@@ -32,7 +34,9 @@ def oracle_paged(kv: "W.PagedKV", storage: np.ndarray) -> oracle.PagedCache:
     return oracle.PagedCache(storage, kv.k_offset, kv.v_offset, kv.dtype, kv.n_kv_heads,
                              kv.head_dim, kv.page_size, kv.num_pages, kv.num_layers,
                              kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride,
-                             bits(kv.page_table), kv.max_pages_per_seq, bits(kv.cache_lengths))
+                             bits(kv.page_table), kv.max_pages_per_seq, bits(kv.cache_lengths),
+                             None if kv.k_scale is None else bits(kv.k_scale),
+                             None if kv.v_scale is None else bits(kv.v_scale))
 
 
 def oracle_cont(kv: "W.ContKV", storage: np.ndarray) -> oracle.ContCache:

@@ -5,7 +5,8 @@ Each mutant is a one-line edit of rope_oracle.c (a flipped sign, swapped cos/sin
 pair partner, a dropped cache length, epsilon outside the root, a sum instead of a mean, a
 dropped weight_offset, a shifted slot, swapped K/V halves, an off-by-one valid length, the
 wrong rotated columns, and in the GEMV + partial RMSNorm: epsilon outside the root, the
-mean over every column, the norm over the tail, a consumed weight_offset).  The copy is built in a temporary directory and the pin suite runs
+mean over every column, the norm over the tail, a consumed weight_offset; and in the FP8
+cache: no saturation, a wrong exponent bias, the scale applied the wrong way).  The copy is built in a temporary directory and the pin suite runs
 against it in a subprocess; the test passes when that run fails.
 """
 import os
@@ -51,6 +52,12 @@ MUTANTS = {
     "gemv norm taken over the tail": (
         "for (int64_t i = 0; i < n_normed; ++i) ss += y[i] * y[i];",
         "for (int64_t i = n - n_normed; i < n; ++i) ss += y[i] * y[i];"),
+    "e4m3 without saturation": ("  if (r > 448.0) r = 448.0;\n", "\n"),
+    "e4m3 exponent bias": ("return sign | (uint8_t)((e - 1 + 7) << 3) | m;",
+                           "return sign | (uint8_t)((e - 1 + 8) << 3) | m;"),
+    "fp8 scale multiplied instead of divided": (
+        "orc_encode(c->dtype, plane ? c->v : c->k, i, v / cache_scale(c, plane));",
+        "orc_encode(c->dtype, plane ? c->v : c->k, i, v * cache_scale(c, plane));"),
     "gemv weight_offset consumed": (
         "orc_encode(dtype, normed_output, i, y[i] * r * orc_decode(dtype, gamma, i));",
         "orc_encode(dtype, normed_output, i, y[i] * r * (orc_decode(dtype, gamma, i) + "

@@ -716,3 +716,77 @@ def test_q_out_in_another_type_is_the_same_value_rounded_once(q_dtype):
         got = qb.reshape(T, 2, 32, 2)
         sp = np.spacing(np.abs(np.stack([y.real, y.imag], -1)).astype(np.float32))
         assert bool(np.all(np.abs(got - np.stack([y.real, y.imag], -1)) <= 0.5 * sp * (1 + 1e-9)))
+
+
+# ------------------------------------------------------------------ FP8 (E4M3) caches --
+
+def _e4m3_roundtrip(vals):
+    """The oracle's codec on float64 values, through a one-column fp8 'cache' of the ragged
+    store's V plane would be indirect; the codec is exported instead."""
+    buf = np.zeros(len(vals), dtype=np.uint8)
+    lib = oracle._load()
+    for i, v in enumerate(vals):
+        lib.orc_encode(3, buf.ctypes.data, i, float(v))
+    back = np.array([lib.orc_decode(3, buf.ctypes.data, i) for i in range(len(vals))])
+    return buf, back
+
+
+def test_e4m3_codec_matches_torch():
+    # every code decodes as torch's float8_e4m3fn does; float32 values inside the finite
+    # range encode as torch rounds them (nearest, ties to even); beyond 448 the reading
+    # saturates (torch's plain cast does not, so those are checked against 448 directly)
+    codes = np.arange(256, dtype=np.uint8)
+    lib = oracle._load()
+    dec = np.array([lib.orc_decode(3, codes.ctypes.data, i) for i in range(256)])
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().double().numpy()
+    assert np.array_equal(np.isnan(dec), np.isnan(ref))
+    assert np.array_equal(dec[~np.isnan(dec)], ref[~np.isnan(ref)])
+    g = torch.Generator().manual_seed(7)
+    x = (torch.randn(4000, generator=g) * torch.exp2(torch.randint(-12, 9, (4000,),
+                                                                   generator=g).float()))
+    x = x[x.abs() < 448].float()
+    # exact midpoints between neighbouring codes, where ties to even decides
+    mids = torch.tensor([(a + b) / 2 for a, b in zip(ref[1:120:7], ref[2:121:7])],
+                        dtype=torch.float32)
+    x = torch.cat([x, mids, -mids])
+    got, _ = _e4m3_roundtrip(x.double().numpy())
+    want = x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, want)
+    sat, back = _e4m3_roundtrip([448.0, 460.0, 1e6, float("inf"), -1e6])
+    assert np.array_equal(back, [448.0, 448.0, 448.0, 448.0, -448.0])
+
+
+def test_fp8_store_holds_the_scaled_value_rounded_once():
+    # an FP8 cache stores e4m3(value / scale) per plane (the reading of the pages' scale_dtype_
+    # and quantization_granularity_: one float32 scale per K / V plane).  V is copied, so its
+    # code is torch's cast of the input divided by an exact power-of-two scale; K is rotated,
+    # so its dequantised value lies within half an e4m3 spacing (plus half a bf16 one) of the
+    # bf16 store's K
+    kw = dict(lengths=[6, 11], cache_lengths=[2, 30], n_q_heads=2, n_kv_heads=2, head_dim=64,
+              page_size=16, rope_dim=64, theta=1e4, interleaved=False, max_seq_len=64)
+    sk, sv = 0.5, 0.0625
+    w8 = W.ragged_store(140, cache_dtype="fp8", kv_scales=(sk, sv), **kw)
+    wb = W.ragged_store(140, **kw)
+    r8, rb = H.oracle_ragged_store(w8), H.oracle_ragged_store(wb)
+    assert r8.err == rb.err == 0
+    assert np.array_equal(r8.q_out, rb.q_out) and np.array_equal(r8.written, rb.written)
+    kv8, kvb = w8.cache, wb.cache
+    shp = (kv8.num_pages, 2, kv8.num_layers, kv8.page_size, 2, 64)
+    rows = H.paged_rows_mask(kv8, r8.written, w8.layer_idx)
+    c8, cb = r8.storage.reshape(shp), rb.storage.reshape(shp)
+    # V plane, written rows: code == torch cast of (input V / sv)
+    T = w8.total_tokens
+    v_in = w8.qkv[:, 4 * 64:6 * 64].float().reshape(T, 2, 64)
+    slots = W.token_slots(kv8, [2, 30], [6, 11])
+    for t, (pg, sl) in enumerate(slots):
+        want = (v_in[t] / sv).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(c8[pg, 1, w8.layer_idx, sl], want)
+    # K plane, written rows: dequantised value close to the bf16 store's
+    kq = torch.from_numpy(c8[:, 0][rows[:, 0]].copy()).view(torch.float8_e4m3fn).double()
+    kq = kq.numpy() * sk
+    kbf = H.values(cb[:, 0][rows[:, 0]], "bf16")
+    e4_ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(kbf) / sk, 2.0 ** -6))) - 3) * sk
+    assert bool(np.all(np.abs(kq - kbf) <= 0.5 * e4_ulp + 0.5 * H.bf16_ulp(kbf) + 1e-12))
+    # bytes outside the written rows are untouched
+    before = H.bits(kv8.storage).reshape(shp)
+    assert np.array_equal(c8[~rows], before[~rows])

@@ -28,7 +28,8 @@ from typing import List, Optional
 
 import torch
 
-TORCH_DTYPES = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
+TORCH_DTYPES = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32,
+                "fp8": torch.float8_e4m3fn}
 PAGE_SENTINEL = -1  # 0xFFFFFFFF once viewed as uint32
 
 
@@ -79,6 +80,9 @@ def random_bits(gen: torch.Generator, n: int, dtype: str = "bf16",
         src = torch.randint(-(1 << 31), (1 << 31) - 1, (min(n, block),), generator=gen,
                             dtype=torch.int32)
         view = torch.float32
+    elif dtype == "fp8":
+        src = torch.randint(0, 256, (min(n, block),), generator=gen, dtype=torch.uint8)
+        view = torch.float8_e4m3fn
     else:
         src = torch.randint(-(1 << 15), 1 << 15, (min(n, block),), generator=gen,
                             dtype=torch.int16)
@@ -113,6 +117,8 @@ class PagedKV:
     page_table: torch.Tensor      # int32 [n_seqs, width], -1 = unused
     cache_lengths: torch.Tensor   # int32 [n_seqs]
     dtype: str = "bf16"
+    k_scale: Optional[torch.Tensor] = None   # float32 [1] each, for an fp8 cache
+    v_scale: Optional[torch.Tensor] = None
 
     @property
     def head_stride(self) -> int:
@@ -151,7 +157,8 @@ class PagedKV:
 def paged_cache(gen: torch.Generator, *, cache_lengths: List[int], lengths: List[int],
                 page_size: int, n_kv_heads: int, head_dim: int, planes: int = 2,
                 num_layers: int = 2, width: Optional[int] = None, spare_pages: int = 2,
-                dtype: str = "bf16", fill: str = "bits") -> PagedKV:
+                dtype: str = "bf16", fill: str = "bits",
+                scales: Optional[tuple] = None) -> PagedKV:
     """A paged cache big enough for every sequence's cache_len + len positions."""
     need = [max(1, math.ceil((c + n) / page_size)) for c, n in zip(cache_lengths, lengths)]
     width = width or max(need)
@@ -168,8 +175,11 @@ def paged_cache(gen: torch.Generator, *, cache_lengths: List[int], lengths: List
         storage = random_bits(gen, n_elem, dtype)
     else:
         storage = normal(gen, (n_elem,), dtype=dtype)
+    ks = vs = None
+    if dtype == "fp8":  # per-plane float32 scales
+        ks, vs = (torch.tensor([x], dtype=torch.float32) for x in (scales or (1.0, 1.0)))
     return PagedKV(storage, planes, num_pages, num_layers, page_size, n_kv_heads, head_dim,
-                   table, torch.tensor(cache_lengths, dtype=torch.int32), dtype)
+                   table, torch.tensor(cache_lengths, dtype=torch.int32), dtype, ks, vs)
 
 
 @dataclass
@@ -254,6 +264,7 @@ def ragged_store(seed: int, *, lengths: List[int], cache_lengths: List[int], n_q
                  weight_offset: float = 0.0, num_layers: int = 2, layer_idx: int = 1,
                  width: Optional[int] = None, rope_col_offset: int = -1,
                  dtype: str = "bf16", row_pad: int = 0, q_out_dtype: Optional[str] = None,
+                 cache_dtype: Optional[str] = None, kv_scales: tuple = (1.0, 1.0),
                  name: str = "") -> RaggedStore:
     gen = generator(seed)
     T = sum(lengths)
@@ -264,7 +275,7 @@ def ragged_store(seed: int, *, lengths: List[int], cache_lengths: List[int], n_q
         qkv = qkv[:, :cols]
     cache = paged_cache(gen, cache_lengths=cache_lengths, lengths=lengths, page_size=page_size,
                         n_kv_heads=n_kv_heads, head_dim=D, num_layers=num_layers, width=width,
-                        dtype=dtype)
+                        dtype=cache_dtype or dtype, scales=kv_scales)
     rope = RopeSpec(freqs_cis(max_seq_len, rope_dim, theta, freq_dtype), freq_dtype,
                     interleaved, rope_col_offset)
     q_out = random_bits(gen, T * n_q_heads * D, q_out_dtype or dtype).view(T, n_q_heads * D)
@@ -315,7 +326,9 @@ def dual_band(seed: int, *, lengths: List[int], cache_lengths: List[int], main_q
               interleaved: bool, max_seq_len: int, x_std: float = 1.0,
               main_eps: float = 1e-6, index_eps: float = 1e-6, weight_offset: float = 0.0,
               num_layers: int = 2, layer_idx: int = 1, dtype: str = "bf16",
-              k_in_place: bool = False, single: bool = False, name: str = "") -> DualBand:
+              k_in_place: bool = False, single: bool = False,
+              main_cache_dtype: Optional[str] = None, index_cache_dtype: Optional[str] = None,
+              kv_scales: tuple = (1.0, 1.0), name: str = "") -> DualBand:
     """k_in_place: the bands' K heads are not read from the input but from the cache slots
     the tokens map to (which hold N(0, x_std) K rows, as if the projection had stored them),
     and V is not stored (the bands' column triples become (q_col, -1, -1)).  single: the
@@ -329,11 +342,12 @@ def dual_band(seed: int, *, lengths: List[int], cache_lengths: List[int], main_q
     inp = normal(gen, (T, cols), std=x_std, dtype=dtype)
     main = paged_cache(gen, cache_lengths=cache_lengths, lengths=lengths,
                        page_size=main_page_size, n_kv_heads=main_kv_heads, head_dim=D,
-                       num_layers=num_layers, width=max_seq_len // main_page_size, dtype=dtype)
+                       num_layers=num_layers, width=max_seq_len // main_page_size,
+                       dtype=main_cache_dtype or dtype, scales=kv_scales)
     index = paged_cache(gen, cache_lengths=cache_lengths, lengths=lengths,
                         page_size=index_page_size, n_kv_heads=index_kv_heads, head_dim=D,
                         planes=1, num_layers=num_layers, width=max_seq_len // index_page_size,
-                        dtype=dtype)
+                        dtype=index_cache_dtype or dtype, scales=kv_scales)
     rope = RopeSpec(freqs_cis(max_seq_len, rope_dim, theta, "f32"), "f32", interleaved)
     gam = tuple(normal(gen, (D,), std=0.1, mean=1.0, dtype=dtype) for _ in range(4))
     q_main_out = random_bits(gen, T * main_q_heads * D, dtype).view(T, main_q_heads * D)
