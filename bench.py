@@ -166,11 +166,13 @@ def positions_ragged(lengths, cache_lengths):
 
 
 def bytes_ragged(w) -> int:
-    """QKV rows read + Q rows written + K and V rows stored + distinct freqs_cis rows."""
+    """QKV rows read + Q rows written + K and V rows stored (in the cache's element size) +
+    distinct freqs_cis rows."""
     D, Hq, Hk = w.cache.head_dim, w.n_q_heads, w.cache.n_kv_heads
-    eb = w.qkv.element_size()
-    row = (Hq + 2 * Hk) * D * eb
-    return w.total_tokens * 2 * row + freqs_bytes(
+    eb, qeb = w.qkv.element_size(), w.q_out.element_size()
+    ceb = w.cache.storage.element_size()
+    per_token = (Hq + 2 * Hk) * D * eb + Hq * D * qeb + 2 * Hk * D * ceb
+    return w.total_tokens * per_token + freqs_bytes(
         w.rope, positions_ragged(w.lengths, w.cache.cache_lengths.tolist()))
 
 
@@ -213,6 +215,7 @@ def bytes_bshd(w) -> int:
 
 WORKLOADS = {
     "llama3_8b_prefill": "rope_split_store_paged_ragged",
+    "llama3_8b_prefill_fp8_cache": "rope_split_store_paged_ragged",
     "per_head_norm": "fused_qk_rmsnorm_rope_paged",
     "per_head_norm_multiply_after_cast": "fused_qk_rmsnorm_rope_paged",
     "dual_band_minimax": "fused_dual_qk_rmsnorm_rope_paged",
@@ -234,7 +237,9 @@ class Case:
 
 def make_workload(name, seed):
     import workloads as W
-    return {"llama3_8b_prefill": W.llama3_8b_prefill, "per_head_norm": W.per_head_norm,
+    return {"llama3_8b_prefill": W.llama3_8b_prefill,
+            "llama3_8b_prefill_fp8_cache": W.llama3_8b_prefill_fp8_cache,
+            "per_head_norm": W.per_head_norm,
             "per_head_norm_multiply_after_cast": W.per_head_norm,
             "dual_band_minimax": W.dual_band_minimax,
             "dual_band_minimax_in_place": W.dual_band_minimax_in_place,
@@ -258,7 +263,9 @@ def make_case(name, seed, dev, w=None, sched=True):
                              None if kv.v_offset is None else storage[kv.v_offset:],
                              d(kv.page_table), d(kv.cache_lengths), kv.n_kv_heads,
                              kv.head_dim, kv.page_size, kv.num_pages, kv.num_layers,
-                             kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride)
+                             kv.page_stride, kv.layer_stride, kv.slot_stride, kv.head_stride,
+                             k_scale=None if kv.k_scale is None else d(kv.k_scale),
+                             v_scale=None if kv.v_scale is None else d(kv.v_scale))
 
     lib = rs.raw_library()
     stream = torch.cuda.current_stream()
@@ -280,7 +287,8 @@ def make_case(name, seed, dev, w=None, sched=True):
     def pinned(t):
         return t.contiguous().pin_memory()
 
-    if name in ("llama3_8b_prefill", "per_head_norm", "per_head_norm_multiply_after_cast"):
+    if name in ("llama3_8b_prefill", "llama3_8b_prefill_fp8_cache", "per_head_norm",
+                "per_head_norm_multiply_after_cast"):
         mbc = 0 if name.endswith("multiply_after_cast") else 1
         w = w or make_workload(name, seed)
         kv = w.cache
@@ -291,8 +299,9 @@ def make_case(name, seed, dev, w=None, sched=True):
         c_f, c_kv = fr.c(), cache.c()
         keep += [c_f, c_kv]
         if w.q_gamma is None:
-            args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
-                    offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), w.layer_idx,
+            args = (qkv.data_ptr(), qkv.stride(0), rs._DTYPE_CODE[qkv.dtype], w.total_tokens,
+                    w.n_q_heads, offs.data_ptr(), offs.shape[0] - 1, ctypes.byref(c_f),
+                    ctypes.byref(c_kv), w.layer_idx,
                     q_out.data_ptr(), q_out.stride(0), -1, c.err.data_ptr(), sched_ptr,
                     stream.cuda_stream)
             c.step = bind(lib.rope_split_store_paged_ragged, args, c.entry_point)
@@ -302,8 +311,9 @@ def make_case(name, seed, dev, w=None, sched=True):
                                                  q_out, c.err, sched=c.sched)
         else:
             qg, kg = d(w.q_gamma), d(w.k_gamma)
-            args = (qkv.data_ptr(), qkv.stride(0), w.total_tokens, w.n_q_heads, offs.data_ptr(),
-                    offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv), qg.data_ptr(),
+            args = (qkv.data_ptr(), qkv.stride(0), -1, w.total_tokens, w.n_q_heads,
+                    offs.data_ptr(), offs.shape[0] - 1, ctypes.byref(c_f), ctypes.byref(c_kv),
+                    qg.data_ptr(),
                     kg.data_ptr(), ctypes.c_float(w.epsilon), ctypes.c_float(w.weight_offset),
                     mbc, w.layer_idx, q_out.data_ptr(), q_out.stride(0), c.err.data_ptr(),
                     sched_ptr, stream.cuda_stream)
@@ -342,7 +352,7 @@ def make_case(name, seed, dev, w=None, sched=True):
         fr = rs.Freqs(d(w.rope.table), w.rope.interleaved)
         mb, ib, c_f = main.c(keep), index.c(keep), fr.c()
         keep += [mb, ib, c_f]
-        args = (ctypes.byref(mb), ctypes.byref(ib), offs.data_ptr(), offs.shape[0] - 1,
+        args = (ctypes.byref(mb), ctypes.byref(ib), -1, offs.data_ptr(), offs.shape[0] - 1,
                 w.total_tokens, ctypes.byref(c_f), ctypes.c_float(w.weight_offset), 1,
                 w.layer_idx, c.err.data_ptr(), sched_ptr, stream.cuda_stream)
         c.step = bind(lib.fused_dual_qk_rmsnorm_rope_paged, args, c.entry_point)
@@ -660,7 +670,9 @@ KERNELS = {"llama3_8b_prefill": "banded_store_kernel<bf16, head_dim 128, no norm
                "banded_store_kernel<bf16, head_dim 128, rmsnorm> (two bands, K in place)",
            "radd_minimax": "radd_kernel<bf16, head_dim 128>",
            "decode_bshd": "bshd_rope_kernel<bf16, head_dim 128>",
-           "mla_kv_a_proj": "gemv_norm_kernel<bf16, 4 rows per CTA>"}
+           "mla_kv_a_proj": "gemv_norm_kernel<bf16, 4 rows per CTA>",
+           "llama3_8b_prefill_fp8_cache":
+               "banded_store_kernel<bf16, head_dim 128, no norm, FP8 cache>"}
 
 
 def summarize(case, sec, peak):

@@ -19,7 +19,7 @@
  *           contiguous blocks of head_dim elements.  All tensor base pointers, row strides
  *           and column offsets must keep every head row 16-byte aligned.
  * Types.    Element types: ROPE_DTYPE_BF16, ROPE_DTYPE_F16, ROPE_DTYPE_F32.  The cache uses
- *           the input's element type.  freqs_cis may be F32, BF16 or F16.  head_dim is 64,
+ *           the input's element type, or ROPE_DTYPE_FP8_E4M3 (see rope_paged_cache_t).  freqs_cis may be F32, BF16 or F16.  head_dim is 64,
  *           128 or 256 (64 or 128 for F32 elements).
  * Math.     Values are widened to float32, normalised and rotated in float32, and rounded
  *           once, to nearest even, into the output type.  V heads and columns that are
@@ -72,7 +72,12 @@ typedef enum {
   ROPE_ERR_CUDA = 3         /* the launch failed (cudaGetLastError() has the cause) */
 } rope_status_t;
 
-typedef enum { ROPE_DTYPE_BF16 = 0, ROPE_DTYPE_F16 = 1, ROPE_DTYPE_F32 = 2 } rope_dtype_t;
+typedef enum {
+  ROPE_DTYPE_BF16 = 0,
+  ROPE_DTYPE_F16 = 1,
+  ROPE_DTYPE_F32 = 2,
+  ROPE_DTYPE_FP8_E4M3 = 3 /* paged caches only: OCP E4M3 codes with per-plane scales */
+} rope_dtype_t;
 
 /* bits of *err_word */
 #define ROPE_DEVERR_ROW_OFFSETS 0x1u /* input_row_offsets is not a partition of [0, T) */
@@ -138,6 +143,14 @@ typedef struct {
   int32_t max_pages_per_seq; /* usable entries of a page-table row */
   const uint32_t *cache_lengths;
   int32_t n_seqs;
+  /* dtype == ROPE_DTYPE_FP8_E4M3: one float32 scale per plane (device pointers); an element
+   * holds the E4M3 code nearest to value / scale (ties to even, saturating at +-448).  The
+   * pages' cache collections carry a scale type and a quantisation granularity without
+   * defining them; this per-plane reading is this library's.  FP8 caches are written by the
+   * three paged stores (K rotated, V copied; not with K updated in place) and rejected
+   * (ROPE_ERR_UNSUPPORTED) by kv_cache_radd.  Ignored for other dtypes (may be NULL). */
+  const float *k_scale;
+  const float *v_scale;
 } rope_paged_cache_t;
 
 /* A continuous-batching K/V cache (ContinuousBatchingKVCacheCollection on the pages).
@@ -185,7 +198,8 @@ typedef struct {
  * out and store K and V into a paged cache (rope_split_store_paged_ragged page: signature,
  * Parameters, Args).
  *   qkv [total_tokens, (n_q_heads + 2*n_kv_heads) * head_dim], row stride qkv_row_stride:
- *       the flat matmul output, columns Q | K | V.
+ *       the flat matmul output, columns Q | K | V, of element type qkv_dtype (rope_dtype_t;
+ *       < 0: the cache's element type, which an FP8 cache does not allow).
  *   input_row_offsets [batch + 1]: sequence b owns rows [offs[b], offs[b+1]).
  *   Row r of sequence b sits at position p = kv->cache_lengths[b] + (r - offs[b]).
  *   Q heads are rotated with freqs_cis row p and written to q_out [total_tokens, n_q_heads *
@@ -195,7 +209,8 @@ typedef struct {
  *   (the page's q_out_dtype parameter, which defaults to dtype): rotated values are rounded
  *   once into it and unrotated columns converted exactly or rounded once. */
 rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_stride,
-                                            int32_t total_tokens, int32_t n_q_heads,
+                                            int32_t qkv_dtype, int32_t total_tokens,
+                                            int32_t n_q_heads,
                                             const uint32_t *input_row_offsets, int32_t batch,
                                             const rope_freqs_t *freqs,
                                             const rope_paged_cache_t *kv, uint32_t layer_idx,
@@ -215,7 +230,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
  * by (gamma + weight_offset); RoPE follows in float32 and the result is rounded once more
  * (the pages name the flag but do not define it; this is the reading taken). */
 rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_stride,
-                                          int32_t total_tokens, int32_t n_q_heads,
+                                          int32_t qkv_dtype, int32_t total_tokens,
+                                          int32_t n_q_heads,
                                           const uint32_t *input_row_offsets, int32_t batch,
                                           const rope_freqs_t *freqs,
                                           const rope_paged_cache_t *kv, const void *q_gamma,
@@ -230,13 +246,15 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
  * bands share input_row_offsets, total_tokens, freqs_cis, weight_offset,
  * multiply_before_cast and layer_idx; each has its own input columns, cache, gammas,
  * epsilon and Q output, and each band's positions come from its own cache_lengths.  The
- * rope geometry must agree across bands: same element type and head_dim in both caches
+ * rope geometry must agree across bands: one input element type input_dtype (< 0: the main
+ * cache's) and the same head_dim in both caches, each cache holding that type or FP8 codes
  * (else ROPE_ERR_INVALID_ARG, the runtime form of the page's compile-time assert).  The
  * result equals fused_qk_rmsnorm_rope_paged on the main band followed by the same on the
  * index band.  index_band may be NULL: the launch then has the main band alone (the general
  * single-band form, e.g. for K updated in place). */
 rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band,
                                                const rope_norm_band_t *index_band,
+                                               int32_t input_dtype,
                                                const uint32_t *input_row_offsets,
                                                int32_t batch, int32_t total_tokens,
                                                const rope_freqs_t *freqs, float weight_offset,
@@ -315,7 +333,8 @@ rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight
  * rope_split_store_paged_ragged with a workspace per stream.  ROPE_ERR_CUDA if the lookup
  * or the clearing fails. */
 rope_status_t rope_split_store_paged_ragged_noalloc(
-    const void *qkv, int64_t qkv_row_stride, int32_t total_tokens, int32_t n_q_heads,
+    const void *qkv, int64_t qkv_row_stride, int32_t qkv_dtype, int32_t total_tokens,
+    int32_t n_q_heads,
     const uint32_t *input_row_offsets, int32_t batch, const rope_freqs_t *freqs,
     const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
     int32_t q_out_dtype, uint32_t *err_word, rope_stream_t stream);

@@ -362,9 +362,12 @@ uint32_t orc_fused_dual_qk_rmsnorm_rope_paged(int32_t dtype, orc_band *main_band
                                               int32_t total_tokens, const orc_rope *rope,
                                               double weight_offset,
                                               int32_t multiply_before_cast, uint32_t layer_idx) {
-  if (main_band->cache->head_dim != index_band->cache->head_dim ||
-      main_band->cache->dtype != index_band->cache->dtype)
-    return ORC_ERR_ARGS;
+  /* one input type and head_dim; each cache holds that type or FP8 codes */
+  if (main_band->cache->head_dim != index_band->cache->head_dim) return ORC_ERR_ARGS;
+  for (int k = 0; k < 2; ++k) {
+    int32_t cd = (k ? index_band : main_band)->cache->dtype;
+    if (cd != dtype && cd != ORC_FP8_E4M3) return ORC_ERR_ARGS;
+  }
   uint32_t e = orc_fused_qk_rmsnorm_rope_paged(dtype, main_band, input_row_offsets, batch,
                                                total_tokens, rope, weight_offset,
                                                multiply_before_cast, layer_idx);

@@ -47,7 +47,8 @@ DEVERR_PAGE_ID, DEVERR_BATCH, DEVERR_TIMEOUT = 0x8, 0x10, 0x20
 SCHED_WORDS = 2
 OVERLAP_OFF, OVERLAP_PDL, OVERLAP_PDL_EARLY_METADATA = 0, 1, 2
 
-_DTYPE_CODE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+_DTYPE_CODE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2,
+               torch.float8_e4m3fn: 3}
 
 if not os.path.exists(LIBRARY_PATH):
     raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
@@ -69,7 +70,7 @@ class c_paged_cache(ctypes.Structure):
                 ("num_layers", _i32), ("page_stride", _i64), ("layer_stride", _i64),
                 ("slot_stride", _i64), ("head_stride", _i64), ("page_table", _vp),
                 ("page_table_stride", _i64), ("max_pages_per_seq", _i32),
-                ("cache_lengths", _vp), ("n_seqs", _i32)]
+                ("cache_lengths", _vp), ("n_seqs", _i32), ("k_scale", _vp), ("v_scale", _vp)]
 
 
 class c_cont_cache(ctypes.Structure):
@@ -89,21 +90,21 @@ class c_norm_band(ctypes.Structure):
 
 _P = ctypes.POINTER
 _lib.rope_split_store_paged_ragged.argtypes = [
-    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _i32,
-    _vp, _vp, _vp]
+    _vp, _i64, _i32, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64,
+    _i32, _vp, _vp, _vp]
 _lib.fused_qk_rmsnorm_rope_paged.argtypes = [
-    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _vp, _vp, _f32, _f32,
-    _i32, _u32, _vp, _i64, _vp, _vp, _vp]
+    _vp, _i64, _i32, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _vp, _vp, _f32,
+    _f32, _i32, _u32, _vp, _i64, _vp, _vp, _vp]
 _lib.fused_dual_qk_rmsnorm_rope_paged.argtypes = [
-    _P(c_norm_band), _P(c_norm_band), _vp, _i32, _i32, _P(c_freqs), _f32, _i32, _u32, _vp,
-    _vp, _vp]
+    _P(c_norm_band), _P(c_norm_band), _i32, _vp, _i32, _i32, _P(c_freqs), _f32, _i32, _u32,
+    _vp, _vp, _vp]
 _lib.qk_rope_bshd_continuous.argtypes = [
     _vp, _i32, _i32, _i32, _i32, _P(c_cont_cache), _P(c_freqs), _u32, _vp, _vp, _vp, _vp]
 _lib.kv_cache_radd.argtypes = [
     _vp, _i64, _i32, _P(c_paged_cache), _vp, _i32, _u32, _u32, _vp, _vp, _vp]
 _lib.rope_split_store_paged_ragged_noalloc.argtypes = [
-    _vp, _i64, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64, _i32,
-    _vp, _vp]
+    _vp, _i64, _i32, _i32, _i32, _vp, _i32, _P(c_freqs), _P(c_paged_cache), _u32, _vp, _i64,
+    _i32, _vp, _vp]
 _lib.matmul_fused_partial_rmsnorm.argtypes = [
     _vp, _vp, _i64, _i32, _i32, _i32, _vp, _f32, _f32, _vp, _i32, _vp, _i32, _vp, _vp, _i64,
     _vp]
@@ -215,6 +216,8 @@ class PagedCache:
     slot_stride: int
     head_stride: int
     max_pages_per_seq: Optional[int] = None
+    k_scale: Optional[torch.Tensor] = None  # float32 [1] each, for an fp8 (E4M3) cache
+    v_scale: Optional[torch.Tensor] = None
 
     def c(self) -> c_paged_cache:
         pt = _idx(self.page_table)
@@ -223,7 +226,8 @@ class PagedCache:
                              self.n_kv_heads, self.head_dim, self.page_size, self.num_pages,
                              self.num_layers, self.page_stride, self.layer_stride,
                              self.slot_stride, self.head_stride, pt.data_ptr(), pt.stride(0),
-                             width, _idx(self.cache_lengths).data_ptr(), pt.shape[0])
+                             width, _idx(self.cache_lengths).data_ptr(), pt.shape[0],
+                             _ptr(self.k_scale), _ptr(self.v_scale))
 
 
 @dataclass
@@ -281,7 +285,8 @@ def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, freqs: Freq
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.rope_split_store_paged_ragged(
-        qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
+        qkv.data_ptr(), _row_stride(qkv), _DTYPE_CODE[qkv.dtype], qkv.shape[0], n_q_heads,
+        offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
         _row_stride(q_out), _DTYPE_CODE[q_out.dtype], _ptr(err_word), _sched(sched),
         _stream(stream)), "rope_split_store_paged_ragged")
@@ -296,7 +301,8 @@ def rope_split_store_paged_ragged_noalloc(qkv, n_q_heads, input_row_offsets, fre
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.rope_split_store_paged_ragged_noalloc(
-        qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
+        qkv.data_ptr(), _row_stride(qkv), _DTYPE_CODE[qkv.dtype], qkv.shape[0], n_q_heads,
+        offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
         _row_stride(q_out), _DTYPE_CODE[q_out.dtype], _ptr(err_word), _stream(stream)),
         "rope_split_store_paged_ragged_noalloc")
@@ -309,7 +315,8 @@ def fused_qk_rmsnorm_rope_paged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.fused_qk_rmsnorm_rope_paged(
-        qkv.data_ptr(), _row_stride(qkv), qkv.shape[0], n_q_heads, offs.data_ptr(),
+        qkv.data_ptr(), _row_stride(qkv), _DTYPE_CODE[qkv.dtype], qkv.shape[0], n_q_heads,
+        offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), q_gamma.data_ptr(),
         k_gamma.data_ptr(), epsilon, weight_offset, int(bool(multiply_before_cast)), layer_idx,
         q_out.data_ptr(), _row_stride(q_out), _ptr(err_word), _sched(sched), _stream(stream)),
@@ -325,7 +332,8 @@ def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: Optional[N
     m, f = main_band.c(keep), freqs.c()
     i = None if index_band is None else ctypes.byref(index_band.c(keep))
     _check(_lib.fused_dual_qk_rmsnorm_rope_paged(
-        ctypes.byref(m), i, offs.data_ptr(), offs.shape[0] - 1, total_tokens,
+        ctypes.byref(m), i, _DTYPE_CODE[main_band.input.dtype], offs.data_ptr(),
+        offs.shape[0] - 1, total_tokens,
         ctypes.byref(f), weight_offset, int(bool(multiply_before_cast)), layer_idx,
         _ptr(err_word), _sched(sched), _stream(stream)), "fused_dual_qk_rmsnorm_rope_paged")
 

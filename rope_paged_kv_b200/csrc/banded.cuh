@@ -25,6 +25,8 @@
 
 #include "common.cuh"
 
+#include <cuda_fp8.h>
+
 namespace rs {
 
 // A CTA is a producer warp, a storer warp and CW consumer warps; the storer keeps LAG
@@ -55,7 +57,31 @@ struct BandDev {
   // Q output in another element type: the consumers write the rotated Q rows, converted,
   // to a stage region at qo_off, from where the storer copies them
   int32_t q_conv, q_dtype, q_eb, qo_off;
+  // FP8 (E4M3) cache: the consumers write K (rotated) and V rows as codes of value / scale
+  // to stage regions at k8_off and v8_off, from where the storer copies them
+  int32_t kv8, k8_off, v8_off;
+  const float *k_scale, *v_scale;
 };
+
+// N float values written to shared memory as N E4M3 codes (nearest, ties to even,
+// saturating at +-448)
+template <int N>
+__device__ __forceinline__ void st_shared_e4m3(unsigned char *p, const float (&x)[N]) {
+  uint32_t w[N / 4];
+#pragma unroll
+  for (int i = 0; i < N / 4; ++i) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i], x[4 * i + 1]),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i + 2], x[4 * i + 3]),
+                                                 __NV_SATFINITE, __NV_E4M3);
+    w[i] = lo | (hi << 16);
+  }
+  if constexpr (N == 8) {
+    st_shared_v2(p, w[0], w[1]);
+  } else {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(w[0]) : "memory");
+  }
+}
 
 // N float values written to shared memory as N elements of type qd (0 bf16, 1 f16, 2 f32),
 // rounded to nearest even
@@ -104,7 +130,8 @@ struct BandedParams {
   int32_t bar_off, meta_off, gamma_off, offs_off, items_off;
 };
 
-// a consumer thread's head row of a token, packed: stage byte offset (18 bits), kind
+// a consumer thread's head row of a token, packed: stage byte offset (18 bits), kind (0 Q,
+// 1 K, 2 V: V rows are items only for an FP8 cache), band, active flag; the kind
 // (0 Q, 1 K), band, active flag
 constexpr uint32_t kItemOffMask = (1u << 18) - 1u;
 constexpr int kItemKindShift = 27;
@@ -243,8 +270,8 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
 template <int CW>
 __host__ __device__ constexpr int pipe_min_ctas() { return CW <= 4 ? ROPE_LIGHT_MIN_CTAS : 2; }
 
-// QCONV: built with the Q-output conversion (only the store without RMSNorm uses it)
-template <typename T, int D, bool NORM, int CW, int LAG, bool QCONV>
+// EXT: built with the extended outputs (a Q output in another element type, FP8 cache rows)
+template <typename T, int D, bool NORM, int CW, int LAG, bool EXT>
 __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     banded_store_kernel(const __grid_constant__ BandedParams p) {
   constexpr int kConsumerWarps = CW;
@@ -481,16 +508,19 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
                        blk, qb);
           }
           const int64_t base = meta[s].kv_base[k];
+          const int CE = (EXT && bd.kv8) ? 1 : EB;  // cache element bytes
+          const uint32_t kcb = (uint32_t)(bd.n_kv * D * CE);
           for (int plane = 0; plane < (bd.n_v ? 2 : 1); ++plane) {
             unsigned char *dst = reinterpret_cast<unsigned char *>(plane ? bd.cache.v : bd.cache.k) +
-                                 base * EB;
-            const unsigned char *src = blk + qb + plane * kb;
+                                 base * CE;
+            const unsigned char *src = (EXT && bd.kv8) ? st + (plane ? bd.v8_off : bd.k8_off)
+                                                       : blk + qb + plane * kb;
             if (bd.kv_contig) {
-              if (kb) bulk_s2g(dst, src, kb);
+              if (kcb) bulk_s2g(dst, src, kcb);
             } else {
               for (int h = 0; h < bd.n_kv; ++h)
-                bulk_s2g(dst + (int64_t)h * bd.cache.head_stride * EB, src + h * D * EB,
-                         (uint32_t)(D * EB));
+                bulk_s2g(dst + (int64_t)h * bd.cache.head_stride * CE, src + h * D * CE,
+                         (uint32_t)(D * CE));
             }
           }
         }
@@ -553,7 +583,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         const int band = j >= p.work0 ? 1 : 0;
         const BandDev &bd = band ? p.band[1] : p.band[0];
         const int r = j - (band ? p.work0 : 0);  // Q heads then K heads: stage rows 0..
-        const int kind = r >= bd.n_q ? 1 : 0;
+        const int kind = r < bd.n_q ? 0 : r < bd.n_q + bd.n_kv ? 1 : 2;
         const uint32_t soff = (uint32_t)(bd.smem_off + r * D * EB);
         w = kItemAct | (uint32_t)band << kItemBandShift | (uint32_t)kind << kItemKindShift | soff;
       }
@@ -563,6 +593,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     float fca[N], fsa[N], fcb[N], fsb[N];
     float ga[N], gb[N];
     int g_sel = -1;
+    float kinv0 = 1.f, kinv1 = 1.f, vinv0 = 1.f, vinv1 = 1.f;  // 1 / scale of FP8 planes
     for (int i = 0;; ++i) {
       const int s = i % p.S;
       if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
@@ -577,6 +608,16 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         if (lane == 0) mbar_arrive(&done[s]);
         break;
       }
+      if (EXT && i == 0) {  // after the producer's wait for the preceding kernels
+        if (p.band[0].kv8) {
+          kinv0 = 1.f / __ldg(p.band[0].k_scale);
+          if (p.band[0].n_v) vinv0 = 1.f / __ldg(p.band[0].v_scale);
+        }
+        if (p.n_bands > 1 && p.band[1].kv8) {
+          kinv1 = 1.f / __ldg(p.band[1].k_scale);
+          if (p.band[1].n_v) vinv1 = 1.f / __ldg(p.band[1].v_scale);
+        }
+      }
       unsigned char *st = stages + (size_t)s * p.stage_bytes;
       const int ok0 = meta[s].ok[0], ok1 = meta[s].ok[1];
       int f_band = -1;
@@ -586,10 +627,11 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         if (!(w & kItemAct)) continue;
         const int band = (w >> kItemBandShift) & 1;
         if (!(band ? ok1 : ok0)) continue;
-        const int kind = (w >> kItemKindShift) & 1;
+        const int kind = (w >> kItemKindShift) & 3;
         const BandDev &bd = band ? p.band[1] : p.band[0];
-        const bool conv = QCONV && kind == 0 && bd.q_conv;  // every lane writes its Q
-        if (!busy && !conv) continue;
+        const bool conv = EXT && kind == 0 && bd.q_conv;  // every lane writes its Q
+        const bool to8 = EXT && kind >= 1 && bd.kv8;       // and its K / V codes
+        if (!busy && !conv && !to8) continue;
         if ((rot_a || rot_b) && f_band != band) {  // this token's table row for the band
           f_band = band;
           const unsigned char *F = st + bd.f_off;
@@ -625,6 +667,20 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         float xa[N], xb[N];
         VT::widen(ld_shared_v4(row + ca * EB), xa);
         VT::widen(ld_shared_v4(row + cb * EB), xb);
+        // the row's first element within the band's [Q | K | V] block
+        const int re = (int)(((w & kItemOffMask) - (uint32_t)bd.smem_off) / EB);
+        if (EXT && kind == 2) {  // a V row of an FP8 cache: scaled and encoded, nothing else
+          const float inv = band ? vinv1 : vinv0;
+#pragma unroll
+          for (int e = 0; e < N; ++e) {
+            xa[e] *= inv;
+            xb[e] *= inv;
+          }
+          unsigned char *vrow = st + bd.v8_off + (re - (bd.n_q + bd.n_kv) * D);
+          st_shared_e4m3<N>(vrow + ca, xa);
+          st_shared_e4m3<N>(vrow + cb, xb);
+          continue;
+        }
         if constexpr (NORM) {
           if (g_sel != band * 2 + kind) {  // gamma does not depend on the token: kept
             g_sel = band * 2 + kind;
@@ -698,10 +754,19 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
           }
         }
         if (conv) {
-          unsigned char *qrow = st + bd.qo_off +
-                                (size_t)(((w & kItemOffMask) - bd.smem_off) / EB) * bd.q_eb;
+          unsigned char *qrow = st + bd.qo_off + (size_t)re * bd.q_eb;
           st_shared_elems<N>(qrow + ca * bd.q_eb, xa, bd.q_dtype);
           st_shared_elems<N>(qrow + cb * bd.q_eb, xb, bd.q_dtype);
+        } else if (to8) {  // a K row of an FP8 cache
+          const float inv = band ? kinv1 : kinv0;
+#pragma unroll
+          for (int e = 0; e < N; ++e) {
+            xa[e] *= inv;
+            xb[e] *= inv;
+          }
+          unsigned char *krow = st + bd.k8_off + (re - bd.n_q * D);
+          st_shared_e4m3<N>(krow + ca, xa);
+          st_shared_e4m3<N>(krow + cb, xb);
         } else {
           if (NORM || rot_a) st_shared_v4(row + ca * EB, VT::narrow(xa));
           if (NORM || rot_b) st_shared_v4(row + cb * EB, VT::narrow(xb));

@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <initializer_list>
 #include <mutex>
 #include <type_traits>
 
@@ -166,8 +167,9 @@ static rope_status_t check_freqs(const rope_freqs_t *f, int dtype, int D, RopeDe
   return ROPE_OK;
 }
 
+// allow_fp8: the cache may hold E4M3 codes (with its scales) instead of the input's type
 static rope_status_t check_paged(const rope_paged_cache_t *c, int dtype, uint32_t layer,
-                                 bool need_v, PagedDev *out) {
+                                 bool need_v, PagedDev *out, bool allow_fp8 = false) {
   if (c == nullptr || c->k == nullptr || c->page_table == nullptr || c->cache_lengths == nullptr)
     return ROPE_ERR_INVALID_ARG;
   if (need_v && c->v == nullptr) return ROPE_ERR_INVALID_ARG;
@@ -175,8 +177,11 @@ static rope_status_t check_paged(const rope_paged_cache_t *c, int dtype, uint32_
       c->max_pages_per_seq < 0 || c->n_seqs < 0 || c->page_table_stride < 0)
     return ROPE_ERR_INVALID_ARG;
   if (layer >= (uint32_t)c->num_layers) return ROPE_ERR_INVALID_ARG;
-  if (c->dtype != dtype) return ROPE_ERR_UNSUPPORTED;
-  const int eb = elem_bytes(dtype);
+  const bool fp8 = c->dtype == ROPE_DTYPE_FP8_E4M3;
+  if (c->dtype != dtype && !(allow_fp8 && fp8)) return ROPE_ERR_UNSUPPORTED;
+  if (fp8 && (c->k_scale == nullptr || (c->v != nullptr && c->v_scale == nullptr)))
+    return ROPE_ERR_INVALID_ARG;
+  const int eb = fp8 ? 1 : elem_bytes(dtype);
   if (!aligned16(c->k) || (c->v && !aligned16(c->v)) || !stride16(c->page_stride, eb) ||
       !stride16(c->layer_stride, eb) || !stride16(c->slot_stride, eb) ||
       !stride16(c->head_stride, eb))
@@ -215,7 +220,7 @@ static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride
     return ROPE_ERR_INVALID_ARG;
   const bool k_inplace = k_col < 0;
   if (norm && (qg == nullptr || kg == nullptr)) return ROPE_ERR_INVALID_ARG;
-  rope_status_t s = check_paged(kv, dtype, layer, v_col >= 0, &bd->cache);
+  rope_status_t s = check_paged(kv, dtype, layer, v_col >= 0, &bd->cache, true);
   if (s != ROPE_OK) return s;
   const int64_t D = kv->head_dim, Hk = kv->n_kv_heads;
   const int eb = elem_bytes(dtype);
@@ -245,6 +250,10 @@ static rope_status_t fill_band(BandDev *bd, const void *input, int64_t in_stride
   bd->eps = eps;
   bd->kv_contig = kv->head_stride == D ? 1 : 0;
   bd->k_inplace = k_inplace ? 1 : 0;
+  bd->kv8 = kv->dtype == ROPE_DTYPE_FP8_E4M3 ? 1 : 0;
+  if (bd->kv8 && k_inplace) return ROPE_ERR_UNSUPPORTED;  // K would have to be decoded
+  bd->k_scale = kv->k_scale;
+  bd->v_scale = kv->v_scale;
   bd->q_conv = q_dtype != dtype ? 1 : 0;
   bd->q_dtype = q_dtype == ROPE_DTYPE_F32 ? 2 : q_dtype == ROPE_DTYPE_F16 ? 1 : 0;
   bd->q_eb = qeb;
@@ -303,10 +312,14 @@ static size_t layout_banded(BandedParams &p, int D, bool norm, const BandedShape
     p.band[k].f_off = (int32_t)off;
     off = round_up(off + p.f_row_bytes, 16);
   }
-  for (int k = 0; k < p.n_bands; ++k) {  // converted Q rows
+  for (int k = 0; k < p.n_bands; ++k) {  // converted Q rows, FP8 K and V rows
     BandDev &bd = p.band[k];
     bd.qo_off = (int32_t)off;
     if (bd.q_conv) off = round_up(off + (int64_t)bd.n_q * D * bd.q_eb, 16);
+    bd.k8_off = (int32_t)off;
+    if (bd.kv8) off = round_up(off + (int64_t)bd.n_kv * D, 16);
+    bd.v8_off = (int32_t)off;
+    if (bd.kv8) off = round_up(off + (int64_t)bd.n_v * D, 16);
   }
   p.stage_bytes = (int32_t)round_up(off, 128);
   int S = (int)(kStageTarget / p.stage_bytes);
@@ -344,19 +357,16 @@ static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStr
 template <typename T, int D, bool NORM>
 static rope_status_t launch_banded_s(ShapeId id, const BandedParams &p, size_t smem,
                                      cudaStream_t st) {
-  if (id == kLight) {
-    if constexpr (!NORM) {
-      if (p.band[0].q_conv)  // Q written in another element type
-        return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag, true>(p, smem, st);
-    }
-    return launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
-  }
-  if (id == kMid) return launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag>(p, smem, st);
-  if constexpr (!NORM) {
-    if (p.band[0].q_conv)  // stages too large for the light ring
-      return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag, true>(p, smem, st);
-  }
-  return launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag>(p, smem, st);
+  // Q in another element type or an FP8 cache: the instantiation with those outputs
+  const bool ext = p.band[0].q_conv || p.band[0].kv8 || (p.n_bands > 1 && p.band[1].kv8);
+  if (id == kLight)
+    return ext ? launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag, true>(p, smem, st)
+               : launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
+  if (id == kMid)
+    return ext ? launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag, true>(p, smem, st)
+               : launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag>(p, smem, st);
+  return ext ? launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag, true>(p, smem, st)
+             : launch_banded_t<T, D, NORM, kHeavyShape.cw, kHeavyShape.lag>(p, smem, st);
 }
 
 template <typename T, bool NORM>
@@ -534,7 +544,8 @@ const char *rope_status_string(rope_status_t s) {
 }
 
 rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_stride,
-                                            int32_t total_tokens, int32_t n_q_heads,
+                                            int32_t qkv_dtype, int32_t total_tokens,
+                                            int32_t n_q_heads,
                                             const uint32_t *input_row_offsets, int32_t batch,
                                             const rope_freqs_t *freqs,
                                             const rope_paged_cache_t *kv, uint32_t layer_idx,
@@ -543,7 +554,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
                                             uint32_t *sched, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
   if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
-  const int dtype = kv->dtype, D = kv->head_dim;
+  // the input's element type: given, or the cache's
+  const int dtype = qkv_dtype >= 0 ? qkv_dtype : kv->dtype, D = kv->head_dim;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
   if (batch > kv->n_seqs || n_q_heads < 0) return ROPE_ERR_INVALID_ARG;
@@ -556,7 +568,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
                 q_out_dtype);
   if (s != ROPE_OK) return s;
   p.n_bands = 1;
-  p.work0 = p.work_total = (int32_t)(Hq + Hk);
+  // head rows the consumers touch: Q and K, and V too when it is encoded for an FP8 cache
+  p.work0 = p.work_total = (int32_t)(Hq + Hk + (p.band[0].kv8 ? Hk : 0));
   p.offs = input_row_offsets;
   p.batch = batch;
   p.T = total_tokens;
@@ -569,7 +582,8 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
 }
 
 rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_stride,
-                                          int32_t total_tokens, int32_t n_q_heads,
+                                          int32_t qkv_dtype, int32_t total_tokens,
+                                          int32_t n_q_heads,
                                           const uint32_t *input_row_offsets, int32_t batch,
                                           const rope_freqs_t *freqs,
                                           const rope_paged_cache_t *kv, const void *q_gamma,
@@ -580,7 +594,8 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
                                           uint32_t *sched, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
   if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
-  const int dtype = kv->dtype, D = kv->head_dim;
+  // the input's element type: given, or the cache's
+  const int dtype = qkv_dtype >= 0 ? qkv_dtype : kv->dtype, D = kv->head_dim;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
   if (batch > kv->n_seqs || n_q_heads < 0) return ROPE_ERR_INVALID_ARG;
@@ -593,7 +608,8 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
                 q_gamma, k_gamma, epsilon, q_out, q_out_row_stride, dtype, layer_idx, true);
   if (s != ROPE_OK) return s;
   p.n_bands = 1;
-  p.work0 = p.work_total = (int32_t)(Hq + Hk);
+  // head rows the consumers touch: Q and K, and V too when it is encoded for an FP8 cache
+  p.work0 = p.work_total = (int32_t)(Hq + Hk + (p.band[0].kv8 ? Hk : 0));
   p.offs = input_row_offsets;
   p.batch = batch;
   p.T = total_tokens;
@@ -608,6 +624,7 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
 
 rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band,
                                                const rope_norm_band_t *index_band,
+                                               int32_t input_dtype,
                                                const uint32_t *input_row_offsets,
                                                int32_t batch, int32_t total_tokens,
                                                const rope_freqs_t *freqs, float weight_offset,
@@ -622,9 +639,12 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
     return ROPE_ERR_INVALID_ARG;
   const rope_paged_cache_t *mc = main_band->cache;
   const rope_paged_cache_t *ic = n_bands == 2 ? index_band->cache : mc;
-  // the rope geometry must agree across the bands
-  if (mc->dtype != ic->dtype || mc->head_dim != ic->head_dim) return ROPE_ERR_INVALID_ARG;
-  const int dtype = mc->dtype, D = mc->head_dim;
+  // the rope geometry must agree across the bands: one input type, one head_dim (each cache
+  // holds that type or FP8 codes)
+  const int dtype = input_dtype >= 0 ? input_dtype : mc->dtype, D = mc->head_dim;
+  if (mc->head_dim != ic->head_dim) return ROPE_ERR_INVALID_ARG;
+  for (const rope_paged_cache_t *c : {mc, ic})
+    if (c->dtype != dtype && c->dtype != ROPE_DTYPE_FP8_E4M3) return ROPE_ERR_INVALID_ARG;
   rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
   if (s != ROPE_OK) return s;
   if (batch > mc->n_seqs || batch > ic->n_seqs) return ROPE_ERR_INVALID_ARG;
@@ -640,7 +660,7 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
                   b->n_q_heads, b->cache, b->q_gamma, b->k_gamma, b->epsilon, b->q_out,
                   b->q_out_row_stride, dtype, layer_idx, true);
     if (s != ROPE_OK) return s;
-    rows[k] = p.band[k].n_q + p.band[k].n_kv;
+    rows[k] = p.band[k].n_q + p.band[k].n_kv + (p.band[k].kv8 ? p.band[k].n_v : 0);
   }
   p.n_bands = n_bands;
   p.work0 = rows[0];
@@ -744,7 +764,8 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
 }
 
 rope_status_t rope_split_store_paged_ragged_noalloc(
-    const void *qkv, int64_t qkv_row_stride, int32_t total_tokens, int32_t n_q_heads,
+    const void *qkv, int64_t qkv_row_stride, int32_t qkv_dtype, int32_t total_tokens,
+    int32_t n_q_heads,
     const uint32_t *input_row_offsets, int32_t batch, const rope_freqs_t *freqs,
     const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
     int32_t q_out_dtype, uint32_t *err_word, rope_stream_t stream) {
@@ -755,7 +776,7 @@ rope_status_t rope_split_store_paged_ragged_noalloc(
   if (cudaMemsetAsync(scratch, 0, ROPE_SCHED_WORDS * sizeof(uint32_t), (cudaStream_t)stream) !=
       cudaSuccess)
     return ROPE_ERR_CUDA;
-  return rope_split_store_paged_ragged(qkv, qkv_row_stride, total_tokens, n_q_heads,
+  return rope_split_store_paged_ragged(qkv, qkv_row_stride, qkv_dtype, total_tokens, n_q_heads,
                                        input_row_offsets, batch, freqs, kv, layer_idx, q_out,
                                        q_out_row_stride, q_out_dtype, err_word, scratch,
                                        stream);

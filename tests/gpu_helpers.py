@@ -22,7 +22,9 @@ def paged(kv: W.PagedKV, storage: torch.Tensor) -> rs.PagedCache:
     return rs.PagedCache(storage[kv.k_offset:], v, to_dev(kv.page_table),
                          to_dev(kv.cache_lengths), kv.n_kv_heads, kv.head_dim, kv.page_size,
                          kv.num_pages, kv.num_layers, kv.page_stride, kv.layer_stride,
-                         kv.slot_stride, kv.head_stride)
+                         kv.slot_stride, kv.head_stride,
+                         k_scale=None if kv.k_scale is None else to_dev(kv.k_scale),
+                         v_scale=None if kv.v_scale is None else to_dev(kv.v_scale))
 
 
 def cont(kv: W.ContKV, storage: torch.Tensor) -> rs.ContCache:

@@ -75,8 +75,8 @@ def test_host_argument_checks_need_no_gpu(rs):
     f = rs.c_freqs(fake, 2, 64, 64, 1, -1)
     kv = rs.c_paged_cache(fake, fake, 0, 2, 64, 16, 8, 2, 4096, 2048, 128, 64, fake, 4, 4,
                           fake, 2)
-    def call(*a):  # the store with q_out in the cache's element type
-        return lib.rope_split_store_paged_ragged(*a[:11], -1, *a[11:])
+    def call(*a):  # the store with the input and q_out in the cache's element type
+        return lib.rope_split_store_paged_ragged(*a[:2], -1, *a[2:11], -1, *a[11:])
     # NULL descriptors / pointers
     assert call(fake, 512, 8, 4, fake, 2, None, ctypes.byref(kv), 1, fake, 256, None, None,
                 None) == rs.ERR_INVALID_ARG
@@ -111,11 +111,11 @@ def test_host_argument_checks_need_no_gpu(rs):
     assert call(fake, 512, 0, 4, fake, 2, ctypes.byref(f), ctypes.byref(kv), 1, fake, 256,
                 None, None, None) == rs.OK
     # the norm op needs both gammas (checked before any launch)
-    assert lib.fused_qk_rmsnorm_rope_paged(fake, 512, 8, 4, fake, 2, ctypes.byref(f),
+    assert lib.fused_qk_rmsnorm_rope_paged(fake, 512, -1, 8, 4, fake, 2, ctypes.byref(f),
                                            ctypes.byref(kv), None, fake, 1e-6, 0.0, 0, 1, fake,
                                            256, None, None, None) == rs.ERR_INVALID_ARG
     # a q_out element type that does not exist
-    assert lib.rope_split_store_paged_ragged(fake, 512, 8, 4, fake, 2, ctypes.byref(f),
+    assert lib.rope_split_store_paged_ragged(fake, 512, -1, 8, 4, fake, 2, ctypes.byref(f),
                                              ctypes.byref(kv), 1, fake, 256, 7, None, None,
                                              None) == rs.ERR_UNSUPPORTED
     # dual band: geometry must agree across bands
@@ -125,7 +125,8 @@ def test_host_argument_checks_need_no_gpu(rs):
                         fake, 128)
     ib = rs.c_norm_band(fake, 1024, 512, 768, -1, 1, ctypes.pointer(kv128), fake, fake, 1e-6,
                         fake, 128)
-    assert lib.fused_dual_qk_rmsnorm_rope_paged(ctypes.byref(mb), ctypes.byref(ib), fake, 2, 8,
+    assert lib.fused_dual_qk_rmsnorm_rope_paged(ctypes.byref(mb), ctypes.byref(ib), -1, fake,
+                                                2, 8,
                                                 ctypes.byref(f), 0.0, 1, 1, None, None,
                                                 None) == rs.ERR_INVALID_ARG
     # radd needs a V plane
@@ -175,3 +176,30 @@ def test_gemv_host_checks_need_no_gpu(rs):
     assert call(*bad) == rs.ERR_INVALID_ARG
     bad = list(args); bad[12] = 7          # unknown element type
     assert call(*bad) == rs.ERR_UNSUPPORTED
+
+
+def test_fp8_cache_host_checks_need_no_gpu(rs):
+    lib = rs.raw_library()
+    fake = 1 << 20
+    f = rs.c_freqs(fake, 2, 64, 64, 1, -1)
+    # an E4M3 cache (dtype 3) needs its scales
+    kv8 = rs.c_paged_cache(fake, fake, 3, 2, 64, 16, 8, 2, 4096, 2048, 128, 64, fake, 4, 4,
+                           fake, 2, None, None)
+    assert lib.rope_split_store_paged_ragged(fake, 512, 0, 8, 4, fake, 2, ctypes.byref(f),
+                                             ctypes.byref(kv8), 1, fake, 256, -1, None, None,
+                                             None) == rs.ERR_INVALID_ARG
+    # an FP8 cache does not say what the input is
+    assert lib.rope_split_store_paged_ragged(fake, 512, -1, 8, 4, fake, 2, ctypes.byref(f),
+                                             ctypes.byref(kv8), 1, fake, 256, -1, None, None,
+                                             None) == rs.ERR_UNSUPPORTED
+    kv8s = rs.c_paged_cache(fake, fake, 3, 2, 64, 16, 8, 2, 4096, 2048, 128, 64, fake, 4, 4,
+                            fake, 2, fake, fake)
+    # radd does not read FP8 caches
+    assert lib.kv_cache_radd(fake, 256, 8, ctypes.byref(kv8s), fake, 2, 0, 1, None, None,
+                             None) == rs.ERR_UNSUPPORTED
+    # K updated in place would have to be decoded: not built
+    mb = rs.c_norm_band(fake, 1024, 0, -1, -1, 2, ctypes.pointer(kv8s), fake, fake, 1e-6,
+                        fake, 128)
+    assert lib.fused_dual_qk_rmsnorm_rope_paged(ctypes.byref(mb), None, 0, fake, 2, 8,
+                                                ctypes.byref(f), 0.0, 1, 1, None, None,
+                                                None) == rs.ERR_UNSUPPORTED

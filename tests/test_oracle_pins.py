@@ -554,6 +554,9 @@ def test_dual_band_geometry_mismatch_is_an_argument_error():
                     max_seq_len=16)
     w.index_cache.head_dim = 32
     assert H.oracle_dual(w).err == oracle.ERR_ARGS
+    w.index_cache.head_dim = 64
+    w.index_cache.dtype = "f16"  # neither the input's type nor FP8 codes
+    assert H.oracle_dual(w).err == oracle.ERR_ARGS
 
 
 # ------------------------------------------------------------------- K updated in place --

@@ -42,7 +42,7 @@ def test_noalloc_store_matches_the_store_with_a_workspace():
         got = G.stage_ragged(w)
         f, c = got.freqs.c(), got.kv.c()
         st = lib.rope_split_store_paged_ragged_noalloc(
-            got.qkv.data_ptr(), got.qkv.stride(0), w.total_tokens, w.n_q_heads,
+            got.qkv.data_ptr(), got.qkv.stride(0), -1, w.total_tokens, w.n_q_heads,
             got.offs.data_ptr(), got.offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c),
             w.layer_idx, got.q_out.data_ptr(), got.q_out.stride(0), -1, got.err.data_ptr(),
             stream.cuda_stream)

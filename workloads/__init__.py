@@ -478,6 +478,18 @@ def tiny_ragged(seed: int = 0) -> RaggedStore:
                        name="tiny ragged store: batch 2, lengths [3,5], 4q/2kv heads, d64")
 
 
+def llama3_8b_prefill_fp8_cache(seed: int = 0) -> RaggedStore:
+    """llama3_8b_prefill storing K and V as E4M3 codes (K scale 0.5, V scale 0.25)."""
+    gen = generator(seed)
+    lengths = uniform_ints(gen, 8, 256, 2048)
+    return ragged_store(seed + 1, lengths=lengths, cache_lengths=[0] * 8, n_q_heads=32,
+                        n_kv_heads=8, head_dim=128, page_size=128, rope_dim=128, theta=5e5,
+                        interleaved=False, max_seq_len=8192, width=64, cache_dtype="fp8",
+                        kv_scales=(0.5, 0.25),
+                        name="Llama-3-8B ragged prefill into an FP8 (E4M3) cache: 32q/8kv "
+                             "heads, d128, batch 8, page 128, half-split RoPE")
+
+
 def llama3_8b_prefill(seed: int = 0) -> RaggedStore:
     """32 Q / 8 KV heads, head_dim 128, batch 8 with lengths U[256, 2048] (about 9k tokens),
     cache_lengths 0, page_size 128, shuffled page table, bf16 QKV ~ N(0, 1), freqs_cis
