@@ -271,6 +271,8 @@ def make_case(name, seed, dev, w=None, sched=True):
     stream = torch.cuda.current_stream()
     c = Case()
     c.name, c.entry_point = name, WORKLOADS[name]
+    c.cache_dtype = {"llama3_8b_prefill_fp8_cache": "fp8_e4m3 (one float32 scale per plane)",
+                     "mla_kv_a_proj": "no cache"}.get(name, "bf16")
     c.err = torch.zeros(1, dtype=torch.int32, device=dev)
     # scheduling workspace of the staged entry points (None: the static token schedule)
     c.sched = rs.sched_workspace(dev) if sched else None
@@ -629,7 +631,7 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, shapes of the named workload)",
         "config": dict({"workload": case.workload.name, "entry_point": case.entry_point,
-                        "tokens_per_rank": case.tokens, "cache_dtype": "bf16",
+                        "tokens_per_rank": case.tokens, "cache_dtype": case.cache_dtype,
                         "l2": f"inputs larger than L2: {n_rep} rotating copies of the "
                               f"workload, launched back to back",
                         "overlap": OVERLAP_NAMES[args.overlap],
