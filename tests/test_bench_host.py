@@ -67,3 +67,31 @@ def test_reference_arm_prints_one_json_line():
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["higher_is_better"] is True
     assert j["steps"] == 2 and j["warmup"] >= 3
+
+
+@pytest.mark.parametrize("n", [1, 3, 7])
+def test_oracle_token_shares_write_what_the_whole_batch_writes(n):
+    # the all-cores CPU baseline splits the batch into token ranges; run one after another
+    # and on threads, the ranges must leave the cache and Q output exactly as one call does
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    from oracle import runners as R
+    w = W.ragged_store(31, lengths=[40, 3, 70], cache_lengths=[5, 60, 0], n_q_heads=4,
+                       n_kv_heads=2, head_dim=64, page_size=16, rope_dim=64, theta=1e4,
+                       interleaved=False, max_seq_len=256)
+    want = R.oracle_ragged_store(w)
+    assert want.err == 0
+    for threaded in (False, True):
+        calls, store, q_out = bench.oracle_token_shares(w, n)
+        if threaded:
+            with ThreadPoolExecutor(n) as ex:
+                errs = list(ex.map(lambda f: f(), calls))
+        else:
+            errs = [f() for f in calls]
+        assert errs == [0] * n
+        assert np.array_equal(store, want.storage)
+        assert np.array_equal(q_out, want.q_out)
