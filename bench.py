@@ -714,6 +714,50 @@ def launch_modes(torch, dev, stream, args, w, peak, reps=300):
     return {"unit": "us per launch", "workload": w.name, **out}
 
 
+# latency-bound entry points: also timed as launches captured in one CUDA graph
+GRAPH_TIMED = ("decode_bshd", "mla_kv_a_proj")
+
+
+def time_graph(torch, name, dev, w, use_sched, n_launch=100, replays=20):
+    """Device time (s) per call of n_launch calls captured in one CUDA graph on a side
+    stream and replayed `replays` times between one pair of events: the calls back to back
+    with no host launch cost between them (each call still a programmatic dependent of the
+    one before).  Returns (seconds per call, None) or (None, the error) if the capture
+    fails."""
+    gs = torch.cuda.Stream(device=dev)
+    try:
+        with torch.cuda.stream(gs):  # the cases' calls are bound to the capture stream
+            cases = [make_case(name, 0, dev, w, use_sched)
+                     for _ in range(REPLICAS_OF.get(name, REPLICAS))]
+            steps = [c.step for c in cases]
+            for i in range(3):  # launch attributes and occupancy queries are made here
+                steps[i % len(steps)]()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gs, capture_error_mode="thread_local"):
+            for i in range(n_launch):
+                steps[i % len(steps)]()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(gs):
+            g.replay()
+            e0.record(gs)
+            for _ in range(replays):
+                g.replay()
+            e1.record(gs)
+        torch.cuda.synchronize()
+        if any(int(c.err.item()) for c in cases):
+            return None, "device error bits set"
+        sec = e0.elapsed_time(e1) / 1e3 / (replays * n_launch)
+        del g
+        return sec, None
+    except Exception as e:  # reported in the JSON line; the other figures stand
+        try:
+            torch.cuda.synchronize()
+        except Exception:
+            pass
+        return None, f"{type(e).__name__}: {e}"[:200]
+
+
 def run_entry_points(torch, dev, stream, headline, peak, use_sched, reps=30):
     """Every other named workload, timed the same way (N=1 only; reported beside the
     headline, not instead of it)."""
@@ -736,6 +780,12 @@ def run_entry_points(torch, dev, stream, headline, peak, use_sched, reps=30):
             cold = time_steps(torch, steps, reps, stream, flush, per_launch=True) / reps / 1e3
             out[name]["us_per_launch_l2_flushed"] = round(cold * 1e6, 2)
             del flush
+        if name in GRAPH_TIMED:
+            sec_g, err = time_graph(torch, name, dev, w, use_sched)
+            out[name]["cuda_graph"] = (
+                {"us_per_launch": round(sec_g * 1e6, 2),
+                 "algorithmic_gbs": round(cases[0].alg_bytes / sec_g / 1e9, 1),
+                 "launches": "100 per graph, 20 replays"} if err is None else {"error": err})
         del cases, steps
         torch.cuda.empty_cache()
     return out

@@ -118,3 +118,13 @@ def test_fp8_cache_with_the_claimed_schedule_and_every_overlap_mode(G):
             check_store(G, w, G.run_ragged(w), r)
     finally:
         rs.set_launch_overlap(before)
+
+
+@pytest.mark.parametrize("q_out_dtype", ["f32", "f16"])
+def test_fp8_cache_with_q_out_in_another_type(G, q_out_dtype):
+    # both extended outputs at once: Q rounded into its own type, K and V as E4M3 codes
+    w = W.ragged_store(54, lengths=[300, 2, 129], cache_lengths=[1, 0, 64], n_q_heads=16,
+                       n_kv_heads=4, head_dim=128, page_size=64, rope_dim=128, theta=1e4,
+                       interleaved=True, max_seq_len=512, q_out_dtype=q_out_dtype,
+                       cache_dtype="fp8", kv_scales=(0.125, 2.0))
+    check_store(G, w, G.run_ragged(w), H.oracle_ragged_store(w, "bf16"))
