@@ -9,18 +9,19 @@
  * ---------------------------------------
  * Memory.   Every pointer argument is a device pointer owned by the caller (destination-
  *           passing style: the caller allocates every output, as the pages' signatures do
- *           for their output tensors).  Descriptor structs (rope_freqs_t, rope_paged_cache_t, ...) live in
- *           host memory and are read only during the call.  The library allocates, frees
- *           and synchronises nothing.
+ *           for their output tensors).  Descriptor structs (rope_freqs_t,
+ *           rope_paged_cache_t, ...) live in host memory and are read only during the call.
+ *           The library allocates, frees and synchronises nothing.
  * Streams.  Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *           default stream).  Work on one stream runs in order, which is what orders a
  *           store after the projection that produced its input.
  * Layout.   Rows are token-major; strides are in ELEMENTS.  Within a row, heads are
  *           contiguous blocks of head_dim elements.  All tensor base pointers, row strides
  *           and column offsets must keep every head row 16-byte aligned.
- * Types.    Element types: ROPE_DTYPE_BF16, ROPE_DTYPE_F16, ROPE_DTYPE_F32.  The cache uses
- *           the input's element type, or ROPE_DTYPE_FP8_E4M3 (see rope_paged_cache_t).  freqs_cis may be F32, BF16 or F16.  head_dim is 64,
- *           128 or 256 (64 or 128 for F32 elements).
+ * Types.    Element types: ROPE_DTYPE_BF16, ROPE_DTYPE_F16, ROPE_DTYPE_F32.  A cache holds
+ *           the input's element type, or ROPE_DTYPE_FP8_E4M3 codes (see rope_paged_cache_t).
+ *           freqs_cis may be F32, BF16 or F16.  head_dim is 64, 128 or 256 (64 or 128 for
+ *           F32 elements).
  * Math.     Values are widened to float32, normalised and rotated in float32, and rounded
  *           once, to nearest even, into the output type.  V heads and columns that are
  *           neither normalised nor rotated are copied bit for bit.
@@ -327,11 +328,10 @@ rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight
  * schedule uses ROPE_SCHED_WORDS words whatever the call's sizes (so no size is too large
  * for it).  The call allocates nothing; it clears those words on `stream` before its
  * launch.  The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  Every call on a device
- * shares the array, so calls that can overlap on the GPU (different streams) race on it and
- * may skip tokens: keep the calls of this entry point in one stream, or use
- * rope_split_store_paged_ragged with a workspace per stream.  ROPE_ERR_CUDA if the lookup
- * or the clearing fails. */
+ * device current).  Every call on a device shares the array, so calls that can overlap on
+ * the GPU (different streams) race on it and may skip tokens: keep the calls of this entry
+ * point in one stream, or use rope_split_store_paged_ragged with a workspace per stream.
+ * ROPE_ERR_CUDA if the lookup or the clearing fails. */
 rope_status_t rope_split_store_paged_ragged_noalloc(
     const void *qkv, int64_t qkv_row_stride, int32_t qkv_dtype, int32_t total_tokens,
     int32_t n_q_heads,

@@ -19,7 +19,10 @@
 //   warp 1, storer:    once the consumers are done with a token, bulk-copies the stage's Q
 //                      block to q_out and its K and V blocks to the cache page, waits until
 //                      the copies have read the stage, and hands the stage back.
-// V rows never enter registers.  The row range of a token is the band concatenation
+// V rows never enter registers, except for an FP8 cache.  The extended-output instantiation
+// (EXT) writes some results to stage regions of their own instead of in place: Q rounded
+// into another element type, and the E4M3 codes of K and V for an FP8 cache; the storer
+// copies those regions out.  The row range of a token is the band concatenation
 // [Q main | K main | V main | Q index | K index | (V index)].
 #pragma once
 
@@ -30,9 +33,9 @@
 namespace rs {
 
 // A CTA is a producer warp, a storer warp and CW consumer warps; the storer keeps LAG
-// bulk-store groups in flight before handing a stage back.  Two shapes are built: a light
-// one (4 consumer warps, more CTAs per SM) for little work per token, and a heavy one
-// (8 consumer warps) for RMSNorm and many heads.
+// bulk-store groups in flight before handing a stage back.  Three shapes are built: a light
+// one (4 consumer warps, more CTAs per SM) for little work per token, and six or eight
+// consumer warps for RMSNorm, many heads and FP8 caches.
 template <int CW>
 __host__ __device__ constexpr int pipe_threads() { return 32 * (CW + 2); }
 
@@ -266,7 +269,7 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
 #define ROPE_LIGHT_MIN_CTAS 2
 #endif
 // resident CTAs per SM the register budget is sized for: the light shape (<= 4 consumer
-// warps) and the heavy one
+// warps) and the six- and eight-warp ones
 template <int CW>
 __host__ __device__ constexpr int pipe_min_ctas() { return CW <= 4 ? ROPE_LIGHT_MIN_CTAS : 2; }
 

@@ -8,9 +8,9 @@
 // them for the R rows.  (Rows too long for shared memory take a register path that loads
 // the chunks directly.)  Each row's dot product is reduced in float32 inside the CTA.
 // Entries past n_normed are rounded and written at once; the entries to be normalised go to
-// the caller's workspace in float32.  The last CTA to finish (a count in the workspace) reads them back, forms their
-// sum of squares in a fixed order, writes x * rsqrt(mean + eps) * gamma and returns the count
-// to zero.  No CTA waits for another.
+// the caller's workspace in float32.  The last CTA to finish (a count in the workspace) reads
+// them back, forms their sum of squares in a fixed order, writes x * rsqrt(mean + eps) *
+// gamma and returns the count to zero.  No CTA waits for another.
 #pragma once
 
 #include "common.cuh"

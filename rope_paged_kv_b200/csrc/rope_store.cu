@@ -3,7 +3,8 @@
 // Kernels (see the headers):
 //   banded.cuh  ragged paged store, optional per-head RMSNorm, one or two bands: persistent
 //               CTAs, a producer warp bulk-copying token rows into a shared-memory ring,
-//               eight consumer warps rotating / normalising and storing;
+//               four, six or eight consumer warps rotating / normalising in place, a
+//               storer warp bulk-copying the results out;
 //   radd.cuh    in-place cache add on the same staging scheme;
 //   bshd.cuh    decode-shaped BSHD RoPE with in-place K, one CTA per token;
 //   gemv_norm.cuh  one-row GEMV + partial RMSNorm, a few rows of W per CTA, the last CTA
