@@ -180,6 +180,14 @@ def _row_stride(t: torch.Tensor) -> int:
     return t.stride(0)
 
 
+def _code(t: torch.Tensor) -> int:
+    """rope_dtype_t of a tensor's element type."""
+    try:
+        return _DTYPE_CODE[t.dtype]
+    except KeyError:
+        raise ValueError(f"unsupported element type {t.dtype}") from None
+
+
 def _idx(t: torch.Tensor) -> torch.Tensor:
     if t.dtype not in (torch.int32, torch.uint32) or not t.is_contiguous():
         raise ValueError("index arrays must be contiguous int32/uint32")
@@ -196,7 +204,7 @@ class Freqs:
         t = self.table
         if t.dim() != 2 or not t.is_contiguous():
             raise ValueError("freqs_cis must be a contiguous [max_seq_len, rope_dim] tensor")
-        return c_freqs(t.data_ptr(), _DTYPE_CODE[t.dtype], t.shape[0], t.shape[1],
+        return c_freqs(t.data_ptr(), _code(t), t.shape[0], t.shape[1],
                        int(bool(self.interleaved)), self.rope_col_offset)
 
 
@@ -222,7 +230,7 @@ class PagedCache:
     def c(self) -> c_paged_cache:
         pt = _idx(self.page_table)
         width = pt.shape[1] if self.max_pages_per_seq is None else self.max_pages_per_seq
-        return c_paged_cache(self.k.data_ptr(), _ptr(self.v), _DTYPE_CODE[self.k.dtype],
+        return c_paged_cache(self.k.data_ptr(), _ptr(self.v), _code(self.k),
                              self.n_kv_heads, self.head_dim, self.page_size, self.num_pages,
                              self.num_layers, self.page_stride, self.layer_stride,
                              self.slot_stride, self.head_stride, pt.data_ptr(), pt.stride(0),
@@ -248,7 +256,7 @@ class ContCache:
 
     def c(self) -> c_cont_cache:
         lt = _idx(self.lookup_table)
-        return c_cont_cache(self.k.data_ptr(), _ptr(self.v), _DTYPE_CODE[self.k.dtype],
+        return c_cont_cache(self.k.data_ptr(), _ptr(self.v), _code(self.k),
                             self.n_kv_heads, self.head_dim, self.num_slots, self.num_layers,
                             self.max_seq_len, self.slot_stride, self.layer_stride,
                             self.pos_stride, self.head_stride, lt.data_ptr(),
@@ -282,13 +290,16 @@ class NormBand:
 def rope_split_store_paged_ragged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
                                   kv: PagedCache, layer_idx, q_out, err_word=None,
                                   stream=None, sched=None) -> None:
+    """Rotate Q and K of a flat ragged QKV batch, write Q to q_out (in q_out's element type)
+    and store K and V into the paged cache `kv` (rope_split_store_paged_ragged page:
+    signature, Parameters, Args).  qkv [T, (Hq + 2 Hk) D]; input_row_offsets [batch + 1]."""
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.rope_split_store_paged_ragged(
-        qkv.data_ptr(), _row_stride(qkv), _DTYPE_CODE[qkv.dtype], qkv.shape[0], n_q_heads,
+        qkv.data_ptr(), _row_stride(qkv), _code(qkv), qkv.shape[0], n_q_heads,
         offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
-        _row_stride(q_out), _DTYPE_CODE[q_out.dtype], _ptr(err_word), _sched(sched),
+        _row_stride(q_out), _code(q_out), _ptr(err_word), _sched(sched),
         _stream(stream)), "rope_split_store_paged_ragged")
 
 
@@ -301,10 +312,10 @@ def rope_split_store_paged_ragged_noalloc(qkv, n_q_heads, input_row_offsets, fre
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.rope_split_store_paged_ragged_noalloc(
-        qkv.data_ptr(), _row_stride(qkv), _DTYPE_CODE[qkv.dtype], qkv.shape[0], n_q_heads,
+        qkv.data_ptr(), _row_stride(qkv), _code(qkv), qkv.shape[0], n_q_heads,
         offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), layer_idx, q_out.data_ptr(),
-        _row_stride(q_out), _DTYPE_CODE[q_out.dtype], _ptr(err_word), _stream(stream)),
+        _row_stride(q_out), _code(q_out), _ptr(err_word), _stream(stream)),
         "rope_split_store_paged_ragged_noalloc")
 
 
@@ -312,10 +323,13 @@ def fused_qk_rmsnorm_rope_paged(qkv, n_q_heads, input_row_offsets, freqs: Freqs,
                                 kv: PagedCache, q_gamma, k_gamma, epsilon, weight_offset,
                                 layer_idx, q_out, multiply_before_cast=True, err_word=None,
                                 stream=None, sched=None) -> None:
+    """Per-head RMSNorm, then RoPE, of Q and K, with the paged store of
+    rope_split_store_paged_ragged: the single-band op that the
+    fused_dual_qk_rms_norm_rope_ragged_paged page fuses twice (its first paragraph)."""
     offs = _idx(input_row_offsets)
     f, c = freqs.c(), kv.c()
     _check(_lib.fused_qk_rmsnorm_rope_paged(
-        qkv.data_ptr(), _row_stride(qkv), _DTYPE_CODE[qkv.dtype], qkv.shape[0], n_q_heads,
+        qkv.data_ptr(), _row_stride(qkv), _code(qkv), qkv.shape[0], n_q_heads,
         offs.data_ptr(),
         offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c), q_gamma.data_ptr(),
         k_gamma.data_ptr(), epsilon, weight_offset, int(bool(multiply_before_cast)), layer_idx,
@@ -327,12 +341,16 @@ def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: Optional[N
                                      input_row_offsets, total_tokens, freqs: Freqs,
                                      weight_offset, layer_idx, multiply_before_cast=True,
                                      err_word=None, stream=None, sched=None) -> None:
+    """The main band and the index band in one launch (fused_dual_qk_rms_norm_rope_ragged_paged
+    page: signature and both paragraphs); index_band None launches the main band alone.  A
+    band with k_col < 0 reads its K heads from the token's cache slot and writes them back
+    there (the key cache updated in place)."""
     offs = _idx(input_row_offsets)
     keep: list = []
     m, f = main_band.c(keep), freqs.c()
     i = None if index_band is None else ctypes.byref(index_band.c(keep))
     _check(_lib.fused_dual_qk_rmsnorm_rope_paged(
-        ctypes.byref(m), i, _DTYPE_CODE[main_band.input.dtype], offs.data_ptr(),
+        ctypes.byref(m), i, _code(main_band.input), offs.data_ptr(),
         offs.shape[0] - 1, total_tokens,
         ctypes.byref(f), weight_offset, int(bool(multiply_before_cast)), layer_idx,
         _ptr(err_word), _sched(sched), _stream(stream)), "fused_dual_qk_rmsnorm_rope_paged")
@@ -340,6 +358,9 @@ def fused_dual_qk_rmsnorm_rope_paged(main_band: NormBand, index_band: Optional[N
 
 def qk_rope_bshd_continuous(q_proj, kv: ContCache, freqs: Freqs, layer_idx, valid_lengths,
                             output, err_word=None, stream=None) -> None:
+    """Continuous-batching decode RoPE: Q of q_proj [B, S, H, D] rotated into output, K
+    rotated in place in its cache slot, for s < valid_lengths[b]
+    (generic_fused_qk_rope_bshd_continuous_batch page: signature, description, Args)."""
     if q_proj.dim() != 4 or not q_proj.is_contiguous() or not output.is_contiguous():
         raise ValueError("q_proj / output must be contiguous [batch, seq_len, heads, head_dim]")
     B, S, H, D = q_proj.shape
@@ -352,6 +373,9 @@ def qk_rope_bshd_continuous(q_proj, kv: ContCache, freqs: Freqs, layer_idx, vali
 
 def kv_cache_radd(a, kv: PagedCache, input_row_offsets, batch_offset, layer_idx,
                   err_word=None, stream=None, sched=None) -> None:
+    """Add a [T, 2 Hk D] into the K (first half of the columns) and V rows of the paged
+    cache at each token's position (generic_kv_cache_radd_dispatch page: description,
+    Args)."""
     offs = _idx(input_row_offsets)
     c = kv.c()
     _check(_lib.kv_cache_radd(
@@ -374,12 +398,17 @@ def matmul_fused_partial_rmsnorm(input, weight, gamma, epsilon, weight_offset, n
                                  unnormed_output, workspace=None, stream=None,
                                  err_word=None) -> None:
     """y = input @ weight.T (input [k], weight [n, k]); normed_output [n_normed] gets the RMS
-    normalised first entries times gamma, unnormed_output [n - n_normed] the rest."""
+    normalised first entries times gamma, unnormed_output [n - n_normed] the rest
+    (MatmulFusedPartialRMSNorm page: description, execute, Args)."""
     n, k = weight.shape
     nn = normed_output.shape[0]
     if unnormed_output.shape[0] != n - nn or input.shape[-1] != k:
         raise ValueError("output sizes must split n; input must have k entries")
-    dtype = _DTYPE_CODE[weight.dtype]
+    dtype = _code(weight)
+    for name, t in (("input", input), ("gamma", gamma), ("normed_output", normed_output),
+                    ("unnormed_output", unnormed_output)):
+        if t is not None and t.numel() and t.dtype != weight.dtype:
+            raise ValueError(f"{name} must have the weight's element type {weight.dtype}")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.matmul_fused_partial_rmsnorm(
         input.data_ptr(), weight.data_ptr(), _row_stride(weight), n, k, 1,

@@ -203,3 +203,24 @@ def test_fp8_cache_host_checks_need_no_gpu(rs):
     assert lib.fused_dual_qk_rmsnorm_rope_paged(ctypes.byref(mb), None, 0, fake, 2, 8,
                                                 ctypes.byref(f), 0.0, 1, 1, None, None,
                                                 None) == rs.ERR_UNSUPPORTED
+
+
+def test_binding_rejects_element_types_before_any_call(rs):
+    # marshalling errors raise in Python before the library is entered (CPU tensors here are
+    # never handed to it)
+    import torch
+    w = torch.zeros(8, 64, dtype=torch.bfloat16)
+    x16 = torch.zeros(64, dtype=torch.float16)
+    out = torch.zeros(8, dtype=torch.bfloat16)
+    g = torch.zeros(8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="input must have the weight's element type"):
+        rs.matmul_fused_partial_rmsnorm(x16, w, g, 1e-6, 0.0, out, out[:0])
+    with pytest.raises(ValueError, match="gamma"):
+        rs.matmul_fused_partial_rmsnorm(torch.zeros(64, dtype=torch.bfloat16), w,
+                                        g.float(), 1e-6, 0.0, out, out[:0])
+    with pytest.raises(ValueError, match="unsupported element type"):
+        rs.matmul_fused_partial_rmsnorm(torch.zeros(64, dtype=torch.int16),
+                                        w.to(torch.int16), g, 1e-6, 0.0, out, out[:0])
+    table = torch.zeros(16, 64, dtype=torch.float64)
+    with pytest.raises(ValueError, match="unsupported element type"):
+        rs.Freqs(table, True).c()
