@@ -16,9 +16,11 @@ of the workload (its own seeded batch: weak scaling, no collective on the data p
 Also printed (same JSON line): `e2e` (the same step through the Python binding with the
 inputs copied from pinned host memory and q_out copied back inside the timed region),
 `roofline` (algorithmic bytes of one launch / mean launch time, against the measured HBM
-copy bandwidth), `cpu_baseline` (the CPU oracle on the host cores), `clocks` (nvidia-smi
-samples during the timed region), and `entry_points` (the other four entry points on their
-named workloads, at N=1).
+copy bandwidth), `cpu_baseline` (the CPU oracle on one host core and on all of them),
+`clocks` (nvidia-smi samples during the timed region), `launch_modes` (the headline under
+every launch-overlap mode and token schedule) and `entry_points` (every other named
+workload through its entry point, at N=1; the latency-bound ones also as launches captured
+in a CUDA graph).
 """
 from __future__ import annotations
 

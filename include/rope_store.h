@@ -200,7 +200,7 @@ typedef struct {
  * Parameters, Args).
  *   qkv [total_tokens, (n_q_heads + 2*n_kv_heads) * head_dim], row stride qkv_row_stride:
  *       the flat matmul output, columns Q | K | V, of element type qkv_dtype (rope_dtype_t;
- *       < 0: the cache's element type, which an FP8 cache does not allow).
+ *       < 0: the cache's element type; with an FP8 cache that is ROPE_ERR_UNSUPPORTED).
  *   input_row_offsets [batch + 1]: sequence b owns rows [offs[b], offs[b+1]).
  *   Row r of sequence b sits at position p = kv->cache_lengths[b] + (r - offs[b]).
  *   Q heads are rotated with freqs_cis row p and written to q_out [total_tokens, n_q_heads *

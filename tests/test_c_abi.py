@@ -1,0 +1,24 @@
+"""include/rope_store.h is a C header and librope_store.so a C library: a plain C99 program
+(tests/c_abi_check.c), compiled with gcc -pedantic -Werror and linked against the library,
+gets the documented answers for calls that return before any CUDA launch."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_c_program_against_the_header_and_library(tmp_path):
+    from rope_paged_kv_b200 import build
+    lib = build.build()
+    exe = tmp_path / "c_abi_check"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), "-o", str(exe),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"),
+                    "-L", os.path.dirname(lib), "-l:" + os.path.basename(lib),
+                    "-Wl,-rpath," + os.path.dirname(lib)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
