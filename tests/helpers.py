@@ -58,7 +58,8 @@ def assert_close_bf16(got_bits: np.ndarray, want_bits: np.ndarray, what: str,
     if extra is not None:
         tol = tol + extra
     same = _as_bits(np.ascontiguousarray(got_bits)) == _as_bits(np.ascontiguousarray(want_bits))
-    bad = ~(same | (np.abs(g - w) <= tol))
+    with np.errstate(invalid="ignore"):  # equal infinities / NaN bits compare as bits
+        bad = ~(same | (np.abs(g - w) <= tol))
     if bad.any():
         idx = np.argwhere(bad)[:8]
         raise AssertionError(
