@@ -6,8 +6,9 @@ pair partner, a dropped cache length, epsilon outside the root, a sum instead of
 dropped weight_offset, a shifted slot, swapped K/V halves, an off-by-one valid length, the
 wrong rotated columns, and in the GEMV + partial RMSNorm: epsilon outside the root, the
 mean over every column, the norm over the tail, a consumed weight_offset; and in the FP8
-cache: no saturation, a wrong exponent bias, the scale applied the wrong way).  The copy is built in a temporary directory and the pin suite runs
-against it in a subprocess; the test passes when that run fails.
+cache: no saturation, a wrong exponent bias, the scale applied the wrong way).  The copy is
+built in a temporary directory and the pin suite runs against it in a subprocess; the test
+passes when that run fails.
 """
 import os
 import shutil
