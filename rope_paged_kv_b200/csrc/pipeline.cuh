@@ -5,7 +5,8 @@
 // multiples), signalled through one "full" mbarrier per stage (transaction-byte counted)
 // and released through one "empty" mbarrier per stage (one arrival per consumer warp).
 // Every wait polls a bounded number of times: a wait that runs out raises an error bit and
-// the CTA leaves its loops instead of hanging.  No cluster multicast is used.
+// the CTA leaves its loops instead of hanging.  Every copy moves between this CTA's own
+// shared memory and this GPU's global memory.
 #pragma once
 
 #include <cuda_runtime.h>
