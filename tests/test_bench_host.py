@@ -64,7 +64,8 @@ def test_reference_arm_prints_one_json_line():
     assert len(lines) == 1
     j = json.loads(lines[0])
     assert j["impl"] == "reference" and j["unit"] == "tokens/s" and j["value"] > 0
-    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
+    assert j["cpu_baseline"]["kind"] == "oracle"
+    assert 1 <= j["cpu_baseline"]["cores"] <= len(os.sched_getaffinity(0))
     assert j["e2e"]["h2d_bytes_per_step"] == 0 and j["higher_is_better"] is True
     assert j["steps"] == 2 and j["warmup"] >= 3
 
