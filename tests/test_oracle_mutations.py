@@ -4,7 +4,8 @@ on the CPU, makes the pin suite fail.
 Each mutant is a one-line edit of rope_oracle.c (a flipped sign, swapped cos/sin, a wrong
 pair partner, a dropped cache length, epsilon outside the root, a sum instead of a mean, a
 dropped weight_offset, a shifted slot, swapped K/V halves, an off-by-one valid length, the
-wrong rotated columns, and in the GEMV + partial RMSNorm: epsilon outside the root, the
+wrong rotated columns, the normalised value rounded after gamma or not at all under
+multiply_before_cast = 0, and in the GEMV + partial RMSNorm: epsilon outside the root, the
 mean over every column, the norm over the tail, a consumed weight_offset; and in the FP8
 cache: no saturation, a wrong exponent bias, the scale applied the wrong way).  The copy is
 built in a temporary directory and the pin suite runs against it in a subprocess; the test
@@ -53,6 +54,12 @@ MUTANTS = {
     "gemv norm taken over the tail": (
         "for (int64_t i = 0; i < n_normed; ++i) ss += y[i] * y[i];",
         "for (int64_t i = n - n_normed; i < n; ++i) ss += y[i] * y[i];"),
+    "multiply after cast rounds after gamma": (
+        "y[d] = multiply_before_cast ? y[d] * r * g : requantize(dtype, y[d] * r) * g;",
+        "y[d] = multiply_before_cast ? y[d] * r * g : requantize(dtype, y[d] * r * g);"),
+    "multiply after cast ignored": (
+        "y[d] = multiply_before_cast ? y[d] * r * g : requantize(dtype, y[d] * r) * g;",
+        "y[d] = y[d] * r * g;"),
     "e4m3 without saturation": ("  if (r > 448.0) r = 448.0;\n", "\n"),
     "e4m3 exponent bias": ("return sign | (uint8_t)((e - 1 + 7) << 3) | m;",
                            "return sign | (uint8_t)((e - 1 + 8) << 3) | m;"),

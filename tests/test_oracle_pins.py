@@ -615,6 +615,38 @@ def test_multiply_after_cast_with_unit_gamma_is_multiply_before_cast():
     assert np.array_equal(a.q_out.reshape(5, Hq * D)[0], b.q_out.reshape(5, Hq * D)[0])
 
 
+def _half(v):
+    """v rounded once to IEEE half (Python's own float packing: nearest, ties to even)."""
+    import struct
+    return np.array([struct.unpack("<e", struct.pack("<e", float(x)))[0] for x in v])
+
+
+def test_multiply_after_cast_rounds_the_normalised_value_before_gamma():
+    """The reading of multiply_before_cast = 0 (parity unpinned: the pages name the flag
+    only), checked against single roundings done by Python's half-precision packing at
+    position 0, where the rotation is the identity: flag 1 gives half(n * g) and flag 0
+    gives half(half(n) * g), with n = x / sqrt(mean(x^2) + eps) in double and
+    g = gamma + weight_offset (both in the element type).  Some elements must differ, so the
+    two orders are told apart."""
+    w = W.ragged_store(115, lengths=[3], cache_lengths=[0], n_q_heads=4, n_kv_heads=1,
+                       head_dim=64, page_size=8, rope_dim=64, theta=1e4, interleaved=False,
+                       max_seq_len=8, norm=True, weight_offset=0.5, x_std=3.0, dtype="f16")
+    a = H.oracle_ragged_store(w, "f16", True)
+    b = H.oracle_ragged_store(w, "f16", False)
+    assert a.err == b.err == 0
+    Hq, D = w.n_q_heads, w.cache.head_dim
+    x = w.qkv[0, :Hq * D].double().numpy().reshape(Hq, D)
+    n = x / np.sqrt((x * x).mean(axis=1, keepdims=True) + w.epsilon)
+    g = w.q_gamma.double().numpy() + _half([w.weight_offset])[0]
+    before = _half((n * g).reshape(-1))
+    after = _half((_half(n.reshape(-1)).reshape(Hq, D) * g).reshape(-1))
+    got_a = H.values(a.q_out.reshape(3, Hq * D)[0], "f16")
+    got_b = H.values(b.q_out.reshape(3, Hq * D)[0], "f16")
+    assert np.array_equal(got_a, before)
+    assert np.array_equal(got_b, after)
+    assert np.any(before != after)
+
+
 # ------------------------------------------------ GEMV + partial RMSNorm (P5) ----------
 
 def _gemv(n, k, n_normed, dtype="f32", seed=120, **kw):
