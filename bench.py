@@ -66,6 +66,9 @@ def parse_args():
     ap.add_argument("--schedule", choices=["claimed", "static"], default="claimed",
                     help="token schedule of the staged kernels: claimed tail (a scheduling "
                          "workspace) or static")
+    ap.add_argument("--profile-range", action="store_true",
+                    help="bracket the timed steps with cudaProfilerStart / Stop, so that a "
+                         "range-replay profiler measures them as one back-to-back range")
     return ap.parse_args()
 
 
@@ -595,7 +598,11 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     t0 = time.time()
+    if args.profile_range:
+        torch.cuda.profiler.start()
     dev_ms = time_steps(torch, steps, K, stream)
+    if args.profile_range:
+        torch.cuda.profiler.stop()
     t1 = time.time()
     barrier()
 
