@@ -133,9 +133,9 @@ struct BandedParams {
   int32_t bar_off, meta_off, gamma_off, offs_off, items_off;
 };
 
-// a consumer thread's head row of a token, packed: stage byte offset (18 bits), kind (0 Q,
-// 1 K, 2 V: V rows are items only for an FP8 cache), band, active flag; the kind
-// (0 Q, 1 K), band, active flag
+// a consumer thread's head row of a token, packed: stage byte offset (18 bits), kind (2 bits
+// from bit 27: 0 Q, 1 K, 2 V; V rows are items only for an FP8 cache), band (bit 29),
+// active flag (bit 30)
 constexpr uint32_t kItemOffMask = (1u << 18) - 1u;
 constexpr int kItemKindShift = 27;
 constexpr int kItemBandShift = 29;
@@ -148,43 +148,6 @@ struct StageMeta {
   int32_t tok;   // the token held by the stage
   int32_t stop;  // no token: the CTA's work is done
 };
-
-// This lane's (cos, sin) for a token from the staged freqs_cis row F (element type fdt).
-// Interleaved: pair e/2 of the lane's vector uses F[fcol + e], F[fcol + e + 1]; fc[e] =
-// fc[e+1] = cos and fs[e] = fs[e+1] = sin.  Half-split: element e uses pair (fcol/2 + e),
-// fc[e] = cos and fs[e] = -sin for the first half (x*c - partner*s) or +sin for the second
-// half (partner*s + x*c).
-template <int N>
-__device__ __forceinline__ void load_lane_freqs(const void *F, int fdt, bool inter, bool first,
-                                                int fcol, float (&fc)[N], float (&fs)[N]) {
-  if (inter) {
-    float f[N];
-    if (fdt == 2)
-      load_freqs<2, N>(F, fcol, f);
-    else if (fdt == 0)
-      load_freqs<0, N>(F, fcol, f);
-    else
-      load_freqs<1, N>(F, fcol, f);
-#pragma unroll
-    for (int e = 0; e < N; e += 2) {
-      fc[e] = fc[e + 1] = f[e];
-      fs[e] = fs[e + 1] = f[e + 1];
-    }
-  } else {
-    float f[2 * N];
-    if (fdt == 2)
-      load_freqs<2, 2 * N>(F, fcol, f);
-    else if (fdt == 0)
-      load_freqs<0, 2 * N>(F, fcol, f);
-    else
-      load_freqs<1, 2 * N>(F, fcol, f);
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-      fc[e] = f[2 * e];
-      fs[e] = first ? -f[2 * e + 1] : f[2 * e + 1];
-    }
-  }
-}
 
 // Load C consecutive 16-byte chunks at `p` (shared memory) into out[0..C).  The lanes of a
 // head-row group read neighbouring C*16-byte runs; issuing chunk (k + rot) % C at step k,

@@ -73,14 +73,6 @@ struct Vec<float> {
   }
 };
 
-// One element of a freqs_cis table of runtime type (0 = bf16, 1 = f16, 2 = f32).
-__device__ __forceinline__ float load_freq(const void *table, int dtype, int64_t i) {
-  if (dtype == 2) return __ldg(reinterpret_cast<const float *>(table) + i);
-  const unsigned short b = __ldg(reinterpret_cast<const unsigned short *>(table) + i);
-  if (dtype == 0) return __uint_as_float(static_cast<uint32_t>(b) << 16);
-  return __half2float(__ushort_as_half(b));
-}
-
 // Streaming (read-once) 16-byte load and plain 16-byte store.
 __device__ __forceinline__ uint4 ld_stream(const void *p) {
   return __ldcs(reinterpret_cast<const uint4 *>(p));

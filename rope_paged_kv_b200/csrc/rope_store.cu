@@ -348,10 +348,10 @@ static size_t layout_banded(BandedParams &p, int D, bool norm, const BandedShape
   return (size_t)round_up(total, 128);
 }
 
-template <typename T, int D, bool NORM, int CW, int LAG, bool QCONV = false>
+template <typename T, int D, bool NORM, int CW, int LAG, bool EXT = false>
 static rope_status_t launch_banded_t(const BandedParams &p, size_t smem, cudaStream_t st) {
   static ShapeCache cache;
-  auto kern = banded_store_kernel<T, D, NORM, CW, LAG, QCONV>;
+  auto kern = banded_store_kernel<T, D, NORM, CW, LAG, EXT>;
   const int occ = resident_ctas(kern, pipe_threads<CW>(), smem, cache);
   if (occ <= 0) return ROPE_ERR_UNSUPPORTED;  // the stage ring does not fit
   const int64_t slots = (int64_t)sm_count() * occ;
