@@ -3,8 +3,10 @@
 Bit-exact: page/slot placement, V copies, columns neither normed nor rotated, every cache
 byte the operation must not touch, the radd sums, the device error bits.  Rotated / normed
 values: |gpu - oracle| <= max(1 ulp of the oracle value in the element type, 1e-3).
-Sizes: the five named workloads at full size (in the launch configuration the benchmark
-uses) plus small cases that span several tiles and ragged tails, and the edge cases.
+Sizes: the five named workloads at full size (with the claimed-tail token schedule the
+benchmark uses, under the default launch-overlap mode; test_gpu_schedule.py shows every mode,
+the benchmark's included, bit-identical) plus small cases that span several tiles and
+ragged tails, and the edge cases.
 """
 import json
 import os
