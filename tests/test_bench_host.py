@@ -96,3 +96,38 @@ def test_oracle_token_shares_write_what_the_whole_batch_writes(n):
         assert errs == [0] * n
         assert np.array_equal(store, want.storage)
         assert np.array_equal(q_out, want.q_out)
+
+
+def test_algorithmic_bytes_of_the_named_workloads():
+    # the per-unit figures the roofline uses, as the design states them: bytes the method
+    # must move per token (QKV read, Q written, K / V written; cache rows read where the op
+    # reads them), plus the distinct freqs_cis rows for the rotating ops
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+
+    def per_token_without_freqs(w, total, freqs_rows_bytes):
+        return (total - freqs_rows_bytes) / w.total_tokens
+
+    w = W.llama3_8b_prefill()
+    fr = len(set(bench.positions_ragged(w.lengths, [0] * 8))) * 128 * 4
+    assert bench.bytes_ragged(w) == 10433 * 24576 + fr
+    assert bench.bytes_ragged(w) == 257437184
+    w8 = W.llama3_8b_prefill_fp8_cache()
+    assert bench.bytes_ragged(w8) == 10433 * (6144 * 2 + 4096 * 2 + 2048 * 1) + fr
+    n = W.per_head_norm()
+    frn = len(set(bench.positions_ragged(n.lengths, n.cache.cache_lengths.tolist()))) * 128 * 4
+    assert per_token_without_freqs(n, bench.bytes_ragged(n), frn) == 40960
+    d = W.dual_band_minimax()
+    frd = len(set(bench.positions_ragged(d.lengths,
+                                         d.main_cache.cache_lengths.tolist()))) * 64 * 4
+    assert per_token_without_freqs(d, bench.bytes_dual(d), frd) == 45568
+    di = W.dual_band_minimax_in_place()
+    assert per_token_without_freqs(di, bench.bytes_dual(di), frd) == 41472
+    r = W.radd_minimax()
+    assert bench.bytes_radd(r) == 32768 * 12288
+    b = W.decode_bshd()
+    frb = len(set(int(c) for c in b.cache.cache_lengths.tolist())) * 128 * 2
+    assert bench.bytes_bshd(b) == 256 * (20736 - 256) + frb
+    g = W.mla_kv_a_proj()
+    assert bench.bytes_gemv(g) == (576 * 7168 + 7168 + 512 + 576) * 2
