@@ -52,7 +52,7 @@ _DTYPE_CODE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2,
 
 if not os.path.exists(LIBRARY_PATH):
     raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
-                      f"`python -m rope_paged_kv_b200.build` (nvcc, sm_100a)")
+                      f"`python rope_paged_kv_b200/build.py` (nvcc, sm_100a)")
 _lib = ctypes.CDLL(LIBRARY_PATH)
 
 _vp, _i32, _i64, _u32, _f32 = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,

@@ -1,6 +1,9 @@
 """Build ``librope_store.so`` (the C-ABI library of include/rope_store.h) for sm_100a.
 
-    python -m rope_paged_kv_b200.build [--force]
+    python rope_paged_kv_b200/build.py [--force]
+
+Run it as a script, or load it from its file: importing the package itself needs the built
+library, so the builder must not be reached through the package.
 """
 from __future__ import annotations
 

@@ -12,8 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def rs():
-    from rope_paged_kv_b200 import build
-    build.build()
+    from conftest import build_library
+    build_library()
     import rope_paged_kv_b200
     return rope_paged_kv_b200
 

@@ -25,8 +25,8 @@ class Recorder:
 
 @pytest.fixture
 def rs(monkeypatch):
-    from rope_paged_kv_b200 import build
-    build.build()
+    from conftest import build_library
+    build_library()
     import rope_paged_kv_b200
     rec = Recorder()
     monkeypatch.setattr(rope_paged_kv_b200, "_lib", rec)

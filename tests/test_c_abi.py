@@ -12,8 +12,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
 def test_c_program_against_the_header_and_library(tmp_path):
-    from rope_paged_kv_b200 import build
-    lib = build.build()
+    from conftest import build_library
+    lib = build_library()
     exe = tmp_path / "c_abi_check"
     subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
                     "-I", os.path.join(ROOT, "include"), "-o", str(exe),
