@@ -16,7 +16,9 @@ Parity status of the functions (what pins each one is stated in the test-suite):
   input's K): pinned.
   multiply_before_cast=0: parity unpinned (the pages name the flag without defining it; the
   reading implemented rounds the normalised value to the element type before the gamma
-  multiply, and only its reduction to the plain op at unit gamma is checked).
+  multiply; what is checked is that the oracle implements that reading: at position 0 it
+  equals single half-precision roundings done by Python's own float packing, and it reduces
+  to the plain op at unit gamma).
   The choice of rotated columns under partial RoPE is a reading of an open point; it is
   pinned only against the reading it implements.
   FP8 (E4M3) caches: the element codec is pinned against torch's float8_e4m3fn; the format
