@@ -290,6 +290,29 @@ def test_partial_rope_is_full_rope_of_the_tail(interleaved):
     assert np.array_equal(got[..., 32:], r_f.q_out.reshape(-1, Hq, 32))
 
 
+@pytest.mark.parametrize("interleaved", [True, False])
+@pytest.mark.parametrize("offset", [0, 16])
+def test_partial_rope_at_another_column_offset(interleaved, offset):
+    """The other reading of partial RoPE (rope_col_offset names the first rotated column):
+    columns [offset, offset + 32) of each head are rotated exactly as a 32-wide head would
+    be, every other column passes through bit for bit."""
+    w_p = _f32_problem(interleaved, rope_dim=32, head_dim=64)
+    w_p.rope.rope_col_offset = offset
+    r_p = H.oracle_ragged_store(w_p, "f32")
+    assert r_p.err == 0
+    Hq = w_p.n_q_heads
+    x = w_p.qkv[:, :Hq * 64].view(-1, Hq, 64)
+    w_f = _f32_problem(interleaved, rope_dim=32, head_dim=32)
+    w_f.qkv[:, :Hq * 32] = x[..., offset:offset + 32].reshape(-1, Hq * 32)
+    w_f.rope.table.copy_(w_p.rope.table)
+    r_f = H.oracle_ragged_store(w_f, "f32")
+    got = r_p.q_out.reshape(-1, Hq, 64)
+    keep = np.ones(64, bool)
+    keep[offset:offset + 32] = False
+    assert np.array_equal(got[..., keep], x[..., keep].numpy())
+    assert np.array_equal(got[..., offset:offset + 32], r_f.q_out.reshape(-1, Hq, 32))
+
+
 # ----------------------------------------------------------------------- RMSNorm pins --
 
 def _norm_problem(gamma_const=None, eps=0.5, wo=0.0, seed=51, interleaved=True):
