@@ -230,3 +230,31 @@ def scatter_slots(kv: W.PagedKV, per_token: np.ndarray, cache_lengths, lengths,
     for i, (page, slot) in enumerate(W.token_slots(kv, list(cache_lengths), list(lengths))):
         out[page, 0, layer_idx, slot] = per_token[i]
     return out
+
+
+# ------------------------------------------------- weight_offset as an element-type scalar --
+
+def exact_norm_rows(seed: int, n_rows: int, head_dim: int) -> torch.Tensor:
+    """[n_rows, head_dim] float64 rows of +-1 and +-3 with exactly 3 * head_dim / 8 threes
+    per row (seeded places and signs).  Every row's mean square is exactly 4, so with
+    epsilon 0 its normalised value x * rsqrt(mean(x^2)) is exactly x / 2, in {+-0.5, +-1.5}:
+    exact in every element type."""
+    gen = W.generator(seed)
+    rows = torch.ones(n_rows, head_dim, dtype=torch.float64)
+    for r in range(n_rows):
+        rows[r, torch.randperm(head_dim, generator=gen)[:3 * head_dim // 8]] = 3.0
+    sign = torch.randint(0, 2, (n_rows, head_dim), generator=gen).double() * 2 - 1
+    return rows * sign
+
+
+def bf16_weight_offset_case(rows: torch.Tensor, weight_offset: float):
+    """For exact_norm_rows `rows`, gamma 0 and epsilon 0 at position 0 (identity rotation):
+    the outputs (rows / 2) * bf16(weight_offset), which are bfloat16 numbers for the offsets
+    the tests use, and the outputs an unrounded weight_offset would give.  Returns (want,
+    unrounded) as bfloat16 tensors; raises if `want` is not exact."""
+    wo_b = torch.tensor(weight_offset, dtype=torch.float64).to(torch.bfloat16).double()
+    want = rows / 2 * wo_b
+    want_b = want.to(torch.bfloat16)
+    assert torch.equal(want_b.double(), want), "the expected outputs must be bf16 numbers"
+    unrounded = (rows / 2 * weight_offset).to(torch.bfloat16)
+    return want_b, unrounded

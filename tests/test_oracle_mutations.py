@@ -3,8 +3,9 @@ on the CPU, makes the pin suite fail.
 
 Each mutant is a one-line edit of rope_oracle.c (a flipped sign, swapped cos/sin, a wrong
 pair partner, a dropped cache length, epsilon outside the root, a sum instead of a mean, a
-dropped weight_offset, a shifted slot, swapped K/V halves, an off-by-one valid length, the
-wrong rotated columns, the normalised value rounded after gamma or not at all under
+dropped weight_offset, a weight_offset left unrounded, a shifted slot, swapped K/V halves,
+an off-by-one valid length, the wrong rotated columns, the normalised value rounded after
+gamma or not at all under
 multiply_before_cast = 0, and in the GEMV + partial RMSNorm: epsilon outside the root, the
 mean over every column, the norm over the tail, a consumed weight_offset; and in the FP8
 cache: no saturation, a wrong exponent bias, the scale applied the wrong way).  The copy is
@@ -35,6 +36,8 @@ MUTANTS = {
                             "double r = 1.0 / sqrt(ss + eps);"),
     "weight_offset dropped": ("double g = orc_decode(dtype, gamma, d) + weight_offset;",
                               "double g = orc_decode(dtype, gamma, d);"),
+    "weight_offset not rounded to the element type": (
+        "double wo = requantize(dtype, weight_offset);", "double wo = weight_offset;"),
     "slot shifted": ("int64_t slot = pos % c->page_size;",
                      "int64_t slot = (pos + 1) % c->page_size;"),
     "radd halves swapped": ("double ak = orc_decode(dtype, a, row * a_row_stride + h * D + d);",

@@ -354,6 +354,48 @@ def test_rmsnorm_weight_offset_one_gamma_zero_is_plain_rmsnorm():
     np.testing.assert_allclose(y, want, rtol=1e-6)
 
 
+def weight_offset_problem(seed, head_dim=64, n_tokens=6):
+    """A bf16 norm store whose every token sits at position 0 (one-token sequences, cache
+    length 0) and whose Q and K head rows are exact_norm_rows, with gamma 0, epsilon 0 and
+    weight_offset 0.3.  Returns the workload and the expected Q and K rows (bf16)."""
+    w = W.ragged_store(seed, lengths=[1] * n_tokens, cache_lengths=[0] * n_tokens,
+                       n_q_heads=2, n_kv_heads=1, head_dim=head_dim, page_size=8,
+                       rope_dim=head_dim, theta=1e4, interleaved=False, max_seq_len=8,
+                       norm=True, epsilon=0.0, weight_offset=0.3)
+    Hq, Hk, D = 2, 1, head_dim
+    rows = H.exact_norm_rows(seed, n_tokens * (Hq + Hk), D)
+    w.qkv[:, :(Hq + Hk) * D] = rows.view(n_tokens, (Hq + Hk) * D).to(torch.bfloat16)
+    w.q_gamma.zero_()
+    w.k_gamma.zero_()
+    want, unrounded = H.bf16_weight_offset_case(rows, w.weight_offset)
+    assert not torch.equal(want, unrounded)  # the case tells the two readings apart
+    want = want.view(n_tokens, Hq + Hk, D)
+    return w, want[:, :Hq], want[:, Hq:]
+
+
+@pytest.mark.parametrize("multiply_before_cast", [True, False])
+def test_rmsnorm_weight_offset_is_a_scalar_of_the_element_type(multiply_before_cast):
+    # fused_dual_qk_rms_norm_rope_ragged_paged, signature: weight_offset is a Scalar[dtype],
+    # so 0.3 acts as bf16(0.3) = 154 * 2^-9.  gamma = 0 and epsilon = 0 on rows whose
+    # normalised value is exactly x / 2 in {+-0.5, +-1.5}, at the identity rotation: every
+    # output is (x / 2) * bf16(0.3), a bf16 number (1.5 * 154 * 2^-9 = 231 * 2^-9), where
+    # the unrounded 1.5 * 0.3 = 0.45 rounds to 230 * 2^-9.  Both orders of the gamma
+    # multiply give it, since x / 2 is exact in bf16.
+    w, want_q, want_k = weight_offset_problem(71)
+    assert w.total_tokens == 6
+    r = H.oracle_ragged_store(w, "bf16", multiply_before_cast)
+    assert r.err == 0
+    Hq, D = w.n_q_heads, w.cache.head_dim
+    H.assert_bits_equal(r.q_out.reshape(-1, Hq, D), H.bits(want_q), "Q rows")
+    kv = w.cache
+    view = torch.from_numpy(r.storage.view(np.int16)).view(torch.bfloat16)
+    view = kv.view6(view)
+    for row, (page, slot) in enumerate(W.token_slots(kv, [0] * w.total_tokens,
+                                                     [1] * w.total_tokens)):
+        H.assert_bits_equal(H.bits(view[page, 0, w.layer_idx, slot]), H.bits(want_k[row]),
+                            f"K row of token {row}")
+
+
 @pytest.mark.parametrize("interleaved", [True, False])
 def test_rmsnorm_comes_before_rope(interleaved):
     # undoing the rotation of the output gives x * rsqrt(ms + eps) * gamma_d, column by
