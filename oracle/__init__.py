@@ -309,7 +309,7 @@ def decode(bits: np.ndarray, dtype: str) -> np.ndarray:
 def encode(values, dtype: str) -> np.ndarray:
     """float64 values -> element bits, rounded once to nearest-even by the oracle's codec."""
     v = np.ascontiguousarray(values, dtype=np.float64)
-    out = np.empty(v.size, dtype=np.float32 if dtype == "f32" else np.uint16)
+    out = np.empty(v.size, dtype={"f32": np.float32, "fp8": np.uint8}.get(dtype, np.uint16))
     lib, code, p = _load(), DTYPES[dtype], _ptr(out)
     flat = v.reshape(-1)
     for i in range(flat.size):
