@@ -326,12 +326,15 @@ rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight
  * Arguments and results are those of rope_split_store_paged_ragged without `sched`: the
  * scheduling workspace is a 256-byte array inside the library, one per device, of which the
  * schedule uses ROPE_SCHED_WORDS words whatever the call's sizes (so no size is too large
- * for it).  The call allocates nothing; it clears those words on `stream` before its
- * launch.  The first call on a device looks up the array's device address (with that
- * device current).  Every call on a device shares the array, so calls that can overlap on
- * the GPU (different streams) race on it and may skip tokens: keep the calls of this entry
- * point in one stream, or use rope_split_store_paged_ragged with a workspace per stream.
- * ROPE_ERR_CUDA if the lookup or the clearing fails. */
+ * for it).  The call allocates nothing; after its argument checks it clears those words
+ * on `stream` and launches (a rejected call, or one with nothing to do, queues nothing).
+ * The first call in a CUDA context looks up the array's device address in that context
+ * (with the device current) and keeps it for later calls in the same context; a context
+ * made later on the device (after a device reset) gets a lookup of its own.  Make that
+ * first call before any stream capture.  Every call on a device shares the array, so calls
+ * that can overlap on the GPU (different streams) race on it and may skip tokens: keep the
+ * calls of this entry point in one stream, or use rope_split_store_paged_ragged with a
+ * workspace per stream.  ROPE_ERR_CUDA if the lookup or the clearing fails. */
 rope_status_t rope_split_store_paged_ragged_noalloc(
     const void *qkv, int64_t qkv_row_stride, int32_t qkv_dtype, int32_t total_tokens,
     int32_t n_q_heads,
@@ -347,6 +350,17 @@ const char *rope_status_string(rope_status_t status);
  * for an unknown mode, leaving the mode as it was. */
 rope_status_t rope_set_launch_overlap(int32_t mode);
 int32_t rope_get_launch_overlap(void);
+
+/* A diagnostic of the failure path, not an operation of the pages: the most polls a
+ * pipeline wait inside the staged kernels (the three paged stores, kv_cache_radd,
+ * matmul_fused_partial_rmsnorm) makes before it gives up, for launches that follow,
+ * process-wide.  A wait that gives up sets ROPE_DEVERR_TIMEOUT, the CTA leaves its loops and
+ * the call returns incomplete.  0 (the default) means about 2^30 polls or 2 s, whichever
+ * ends first; the waits that let a CTA's in-flight copies land before it exits keep that
+ * default whatever is set here.  A small limit (1) makes waits run out in normal operation:
+ * a test of the timeout path. */
+rope_status_t rope_set_wait_limit(uint32_t polls);
+uint32_t rope_get_wait_limit(void);
 
 #ifdef __cplusplus
 }

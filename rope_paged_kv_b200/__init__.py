@@ -111,9 +111,13 @@ _lib.matmul_fused_partial_rmsnorm.argtypes = [
 _lib.rope_set_launch_overlap.argtypes = [_i32]
 _lib.rope_get_launch_overlap.argtypes = []
 _lib.rope_get_launch_overlap.restype = _i32
+_lib.rope_set_wait_limit.argtypes = [_u32]
+_lib.rope_get_wait_limit.argtypes = []
+_lib.rope_get_wait_limit.restype = _u32
 for _f in ("rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
            "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd",
            "rope_set_launch_overlap", "rope_split_store_paged_ragged_noalloc",
+           "rope_set_wait_limit",
            "matmul_fused_partial_rmsnorm"):
     getattr(_lib, _f).restype = ctypes.c_int
 _lib.rope_status_string.argtypes = [ctypes.c_int]
@@ -172,6 +176,16 @@ def set_launch_overlap(mode: int) -> None:
 
 def get_launch_overlap() -> int:
     return int(_lib.rope_get_launch_overlap())
+
+
+def set_wait_limit(polls: int) -> None:
+    """The most polls a pipeline wait makes before it gives up (0: the default), for the
+    launches that follow (process-wide): a diagnostic of the timeout path."""
+    _check(_lib.rope_set_wait_limit(int(polls)), "rope_set_wait_limit")
+
+
+def get_wait_limit() -> int:
+    return int(_lib.rope_get_wait_limit())
 
 
 def _row_stride(t: torch.Tensor) -> int:

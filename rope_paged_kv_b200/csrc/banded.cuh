@@ -30,6 +30,8 @@
 
 #include <cuda_fp8.h>
 
+#include <type_traits>
+
 namespace rs {
 
 // A CTA is a producer warp, a storer warp and CW consumer warps; the storer keeps LAG
@@ -66,10 +68,10 @@ struct BandDev {
   const float *k_scale, *v_scale;
 };
 
-// N float values written to shared memory as N E4M3 codes (nearest, ties to even,
+// N float values written at shared address a as N E4M3 codes (nearest, ties to even,
 // saturating at +-448)
 template <int N>
-__device__ __forceinline__ void st_shared_e4m3(unsigned char *p, const float (&x)[N]) {
+__device__ __forceinline__ void sts_e4m3(uint32_t a, const float (&x)[N]) {
   uint32_t w[N / 4];
 #pragma unroll
   for (int i = 0; i < N / 4; ++i) {
@@ -80,21 +82,21 @@ __device__ __forceinline__ void st_shared_e4m3(unsigned char *p, const float (&x
     w[i] = lo | (hi << 16);
   }
   if constexpr (N == 8) {
-    st_shared_v2(p, w[0], w[1]);
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(w[0]), "r"(w[1]) : "memory");
   } else {
-    asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(w[0]) : "memory");
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(w[0]) : "memory");
   }
 }
 
-// N float values written to shared memory as N elements of type qd (0 bf16, 1 f16, 2 f32),
-// rounded to nearest even
+// N float values written at shared address a as N elements of type qd (0 bf16, 1 f16,
+// 2 f32), rounded to nearest even
 template <int N>
-__device__ __forceinline__ void st_shared_elems(unsigned char *p, const float (&x)[N], int qd) {
+__device__ __forceinline__ void sts_elems(uint32_t a, const float (&x)[N], int qd) {
   if (qd == 2) {
 #pragma unroll
     for (int k = 0; k < N; k += 4)
-      st_shared_v4(p + k * 4, make_uint4(__float_as_uint(x[k]), __float_as_uint(x[k + 1]),
-                                         __float_as_uint(x[k + 2]), __float_as_uint(x[k + 3])));
+      sts_v4(a + k * 4, make_uint4(__float_as_uint(x[k]), __float_as_uint(x[k + 1]),
+                                   __float_as_uint(x[k + 2]), __float_as_uint(x[k + 3])));
     return;
   }
   uint32_t w[N / 2];
@@ -109,10 +111,78 @@ __device__ __forceinline__ void st_shared_elems(unsigned char *p, const float (&
     }
   }
   if constexpr (N == 8) {
-    st_shared_v4(p, make_uint4(w[0], w[1], w[2], w[3]));
+    sts_v4(a, make_uint4(w[0], w[1], w[2], w[3]));
   } else {
-    st_shared_v2(p, w[0], w[1]);
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(w[0]), "r"(w[1]) : "memory");
   }
+}
+
+__device__ __forceinline__ uint32_t e4m3_code(float x) {
+  return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3)));
+}
+
+// The E4M3 code of v / s rounded exactly as one rounding of the true quotient would
+// (nearest, ties to even, saturating at +-448), for finite v and a finite scale s whose
+// rounded reciprocal inv is a normal float.  q = v * inv lies within two float32 ulps of
+// v / s, so the codes of q moved two ulps down and up in magnitude agree (and are the
+// answer) unless a rounding boundary m of the E4M3 grid lies between them; then the sign
+// of v - m * s, which one fused multiply-add gives exactly, says on which side of m the
+// quotient lies (zero: it is m, and the tie goes to the even code).
+__device__ __forceinline__ uint32_t e4m3_exact(float v, float inv, float s) {
+  const float q = v * inv;
+  const uint32_t b = __float_as_uint(q), mag = b & 0x7fffffffu, sgn = b & 0x80000000u;
+  if (mag >= 0x7f7ffffeu) return e4m3_code(q);  // saturates (or is not finite) either way
+  const float lo = __uint_as_float((mag < 2u ? 0u : mag - 2u) | sgn);
+  const float hi = __uint_as_float((mag + 2u) | sgn);
+  const uint32_t pr = __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t cl = pr & 0xffu, ch = pr >> 8;
+  if (cl == ch) return cl;
+  const float m = 0.5f * (e4m3_value(cl) + e4m3_value(ch));  // exact: a 5-bit number
+  const float r = fmaf(-m, s, v);
+  if (r == 0.f) return e4m3_code(m);
+  const bool above = (r > 0.f) == (s > 0.f);  // v / s > m
+  // ch has the larger magnitude: the larger value when q >= 0
+  return above == (sgn == 0u) ? ch : cl;
+}
+
+// E4M3 codes of v0..v3 / s as one word (code i in byte i), each rounded exactly once as
+// e4m3_exact does: the codes of the four quotients moved two ulps down and up in magnitude
+// come from two packed conversions each, and agree as words unless a rounding boundary lies
+// between them for some value (or a value is not finite or saturates), which sends that
+// word through e4m3_exact value by value.
+__device__ __forceinline__ uint32_t e4m3_exact4(float v0, float v1, float v2, float v3,
+                                                 float inv, float s) {
+  const float v[4] = {v0, v1, v2, v3};
+  uint32_t lo[4], hi[4];
+  bool edge = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t b = __float_as_uint(v[i] * inv), mag = b & 0x7fffffffu;
+    lo[i] = mag < 2u ? b : b - 2u;  // sign and magnitude: two ulps toward zero
+    hi[i] = b + 2u;                 // and away from it
+    edge |= mag >= 0x7f7ffffeu;
+  }
+  const uint32_t cl = __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(lo[0]),
+                                                           __uint_as_float(lo[1])),
+                                               __NV_SATFINITE, __NV_E4M3) |
+                      (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(lo[2]),
+                                                                     __uint_as_float(lo[3])),
+                                                         __NV_SATFINITE, __NV_E4M3)
+                          << 16;
+  const uint32_t ch = __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(hi[0]),
+                                                           __uint_as_float(hi[1])),
+                                               __NV_SATFINITE, __NV_E4M3) |
+                      (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(hi[2]),
+                                                                     __uint_as_float(hi[3])),
+                                                         __NV_SATFINITE, __NV_E4M3)
+                          << 16;
+  if (cl == ch && !edge) return cl;
+  return e4m3_exact(v[0], inv, s) | e4m3_exact(v[1], inv, s) << 8 |
+         e4m3_exact(v[2], inv, s) << 16 | e4m3_exact(v[3], inv, s) << 24;
 }
 
 struct BandedParams {
@@ -128,6 +198,7 @@ struct BandedParams {
   uint32_t *err;
   float weight_offset;
   int32_t mbc;  // multiply_before_cast: 0 rounds the normalised value before the gamma multiply
+  uint32_t wait_polls;  // the most polls of a pipeline wait (drains keep kSpinLimit)
   // dynamic shared memory layout
   int32_t S, stage_bytes, f_row_bytes, staged, elem_bytes;
   int32_t bar_off, meta_off, gamma_off, offs_off, items_off;
@@ -148,6 +219,13 @@ struct StageMeta {
   int32_t tok;   // the token held by the stage
   int32_t stop;  // no token: the CTA's work is done
 };
+
+// Whether the per-lane table and gamma loads rotate their chunk order so that the lanes of
+// a quarter-warp hit distinct banks (undone with selects), or read in plain order.
+#ifndef ROPE_LDS_ROTATE
+#define ROPE_LDS_ROTATE 1
+#endif
+constexpr bool kLdsRotate = ROPE_LDS_ROTATE != 0;
 
 // Load C consecutive 16-byte chunks at `p` (shared memory) into out[0..C).  The lanes of a
 // head-row group read neighbouring C*16-byte runs; issuing chunk (k + rot) % C at step k,
@@ -187,7 +265,7 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
     constexpr int C = M / 4;           // 16-byte chunks per lane
     constexpr int LP = 32 / M > 0 ? 32 / M : 1;  // lanes sharing one 128-byte line
     uint4 c[C];
-    lds_chunks<C>(F + col * 4, (gl / LP) % C, c);
+    lds_chunks<C>(F + col * 4, kLdsRotate ? (gl / LP) % C : 0, c);
 #pragma unroll
     for (int k = 0; k < C; ++k) {
       f[4 * k] = __uint_as_float(c[k].x);
@@ -201,7 +279,7 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
     if constexpr (M >= 8) {
       constexpr int LP = 64 / M;
       uint4 c[C];
-      lds_chunks<C>(F + col * 2, (gl / LP) % C, c);
+      lds_chunks<C>(F + col * 2, kLdsRotate ? (gl / LP) % C : 0, c);
 #pragma unroll
       for (int k = 0; k < C; ++k) {
         w[4 * k] = c[k].x;
@@ -228,17 +306,353 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
   }
 }
 
-#ifndef ROPE_LIGHT_MIN_CTAS
-#define ROPE_LIGHT_MIN_CTAS 2
+// Head rows a consumer thread takes at once (overlapping their dependency chains), within
+// the register budget of the shape: light CTAs run three to an SM, the others two (a
+// four-warp norm CTA then has about 168 registers a thread).
+#ifndef ROPE_CHUNK_ROWS_NORM
+#define ROPE_CHUNK_ROWS_NORM 3
 #endif
-// resident CTAs per SM the register budget is sized for: the light shape (<= 4 consumer
-// warps) and the six- and eight-warp ones
-template <int CW>
-__host__ __device__ constexpr int pipe_min_ctas() { return CW <= 4 ? ROPE_LIGHT_MIN_CTAS : 2; }
+#ifndef ROPE_CHUNK_ROWS_NORM4
+#define ROPE_CHUNK_ROWS_NORM4 4
+#endif
+#ifndef ROPE_CHUNK_ROWS_ROPE
+#define ROPE_CHUNK_ROWS_ROPE 1
+#endif
+#ifndef ROPE_CHUNK_ROWS_8W
+#define ROPE_CHUNK_ROWS_8W 1
+#endif
+template <int CW, bool NORM>
+__host__ __device__ constexpr int chunk_rows() {
+  return CW >= 8 ? ROPE_CHUNK_ROWS_8W
+                 : !NORM ? ROPE_CHUNK_ROWS_ROPE
+                         : CW <= 4 ? ROPE_CHUNK_ROWS_NORM4 : ROPE_CHUNK_ROWS_NORM;
+}
+
+// M consecutive float32 values from shared address a (16-byte aligned), read bank-conflict
+// free across the lanes of a group (gl = lane index inside the group), as lds_freqs does.
+template <int M>
+__device__ __forceinline__ void lds_f32(uint32_t a, int gl, float (&f)[M]) {
+  constexpr int C = M / 4;
+  constexpr int LP = 32 / M > 0 ? 32 / M : 1;
+  const int rot = kLdsRotate ? (gl / LP) % C : 0;
+  uint4 t[C], c[C];
+#pragma unroll
+  for (int k = 0; k < C; ++k) t[k] = lds_v4(a + ((k + rot) % C) * 16);
+#pragma unroll
+  for (int k = 0; k < C; ++k) c[k] = t[k];
+  if constexpr (C >= 2) {
+    if (rot & 1) {
+#pragma unroll
+      for (int k = 0; k < C; ++k) c[(k + 1) % C] = t[k];
+#pragma unroll
+      for (int k = 0; k < C; ++k) t[k] = c[k];
+    }
+  }
+  if constexpr (C >= 4) {
+    if (rot & 2) {
+#pragma unroll
+      for (int k = 0; k < C; ++k) c[(k + 2) % C] = t[k];
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < C; ++k) {
+    f[4 * k] = __uint_as_float(c[k].x);
+    f[4 * k + 1] = __uint_as_float(c[k].y);
+    f[4 * k + 2] = __uint_as_float(c[k].z);
+    f[4 * k + 3] = __uint_as_float(c[k].w);
+  }
+}
+
+// What a consumer lane owns of every head row: its two vectors (first columns ca, cb; table
+// columns fa, fb), whether each is rotated, the layout and the lane's group.
+struct ConsumerLane {
+  int li, ca, cb, fa, fb, fdt;
+  bool inter, rot_a, rot_b;
+  unsigned gmask;
+};
+
+// Two float values rounded to the element type T (nearest even) and widened back.
+template <typename T>
+__device__ __forceinline__ float2 round2(float2 v) {
+  if constexpr (sizeof(T) == 4) {
+    return v;
+  } else if constexpr (std::is_same<T, __half>::value) {
+    return __half22float2(__floats2half2_rn(v.x, v.y));
+  } else {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v.x, v.y);
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(&h);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+}
+
+// The token's (cos, sin) for a consumer lane.  Interleaved, pair k of vector a: (c[k],
+// s[k]); of vector b: (c2[k], s2[k]).  Half-split, as float2 over the lane's N pairs: P[k] =
+// (c_2k, c_2k+1), Q = (s_2k, s_2k+1), R = -Q.
+template <int N, bool INTER>
+struct LaneFreqs;
+template <int N>
+struct LaneFreqs<N, true> {
+  float c[N / 2], s[N / 2], c2[N / 2], s2[N / 2];
+};
+template <int N>
+struct LaneFreqs<N, false> {
+  float2 P[N / 2], Q[N / 2], R[N / 2];
+};
+
+template <int N, bool INTER>
+__device__ __forceinline__ void load_lane_freqs(LaneFreqs<N, INTER> &fr, const ConsumerLane &cl,
+                                                const unsigned char *F) {
+  if constexpr (INTER) {
+    float f[N];
+    if (cl.rot_a) {
+      lds_freqs<N>(F, cl.fdt, cl.fa, cl.li, f);
+#pragma unroll
+      for (int k = 0; k < N / 2; ++k) {
+        fr.c[k] = f[2 * k];
+        fr.s[k] = f[2 * k + 1];
+      }
+    }
+    if (cl.rot_b) {
+      lds_freqs<N>(F, cl.fdt, cl.fb, cl.li, f);
+#pragma unroll
+      for (int k = 0; k < N / 2; ++k) {
+        fr.c2[k] = f[2 * k];
+        fr.s2[k] = f[2 * k + 1];
+      }
+    }
+  } else if (cl.rot_a) {
+    float f[2 * N];
+    lds_freqs<2 * N>(F, cl.fdt, cl.fa, cl.li, f);
+#pragma unroll
+    for (int k = 0; k < N / 2; ++k) {
+      fr.P[k] = make_float2(f[4 * k], f[4 * k + 2]);
+      fr.Q[k] = make_float2(f[4 * k + 1], f[4 * k + 3]);
+      fr.R[k] = make_float2(-f[4 * k + 1], -f[4 * k + 3]);
+    }
+  }
+}
+
+// RoPE of a lane's two vectors of one head row.
+template <int H2, bool INTER>
+__device__ __forceinline__ void rotate_lane(const LaneFreqs<2 * H2, INTER> &fr,
+                                            const ConsumerLane &cl, float2 (&xa)[H2],
+                                            float2 (&xb)[H2]) {
+  if constexpr (INTER) {
+    if (cl.rot_a)
+#pragma unroll
+      for (int k = 0; k < H2; ++k) {  // (a, b) -> (a c - b s, a s + b c)
+        const float a = xa[k].x, b = xa[k].y;
+        xa[k] = make_float2(fmaf(a, fr.c[k], -b * fr.s[k]), fmaf(a, fr.s[k], b * fr.c[k]));
+      }
+    if (cl.rot_b)
+#pragma unroll
+      for (int k = 0; k < H2; ++k) {
+        const float a = xb[k].x, b = xb[k].y;
+        xb[k] = make_float2(fmaf(a, fr.c2[k], -b * fr.s2[k]), fmaf(a, fr.s2[k], b * fr.c2[k]));
+      }
+  } else if (cl.rot_a) {
+    // pair element e of vector a with element e of vector b
+#pragma unroll
+    for (int k = 0; k < H2; ++k) {
+      const float2 a = xa[k], b = xb[k];
+      xa[k] = __ffma2_rn(b, fr.R[k], __fmul2_rn(a, fr.P[k]));
+      xb[k] = __ffma2_rn(a, fr.Q[k], __fmul2_rn(b, fr.P[k]));
+    }
+  }
+}
+
+// Where a band's rows go in the extended-output instantiation: Q rows rounded into q_dtype
+// at shared address qo (when q_conv), K rows as E4M3 codes of value * kinv at k8 (when kv8),
+// others back in place; row r of the band's block sits at blk + r * D * element size.
+struct BandOut {
+  uint32_t blk, qo, k8;
+  int q_conv, q_dtype, q_eb, kv8, n_q;
+  float kinv;
+};
+
+// gamma + weight_offset of a lane's columns for one row kind (the shared address of its
+// gamma row), kept in registers across rows while the kind does not change
+template <int N>
+struct LaneGamma {
+  uint32_t addr;
+  float a[N], b[N];
+};
+
+// J head rows of a staged token, listed at it[0], it[stride], ...: optionally normalised
+// (per-head RMSNorm with the gamma rows at shared addresses gq / gk for Q / K rows), then
+// rotated with the token's table row F (INTER: the interleaved layout), written back in
+// place.  The J rows' dependency chains are interleaved.  EF: `fr` holds the table row
+// already; else it is read here, after the norm (so that it and the gammas are never live
+// together).  KG: `lg` keeps the gamma last read across calls; else gammas are read per
+// chunk.  EXT: outputs as `bo` says.
+template <int J, typename T, int D, bool NORM, int L, bool INTER, bool EXT, bool EF, bool KG>
+__device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t *it, int stride,
+                                          uint32_t st, uint32_t gq, uint32_t gk, float eps,
+                                          int mbc, const unsigned char *F,
+                                          LaneFreqs<Vec<T>::N, INTER> &fr,
+                                          LaneGamma<Vec<T>::N> &lg, const BandOut &bo) {
+  using VT = Vec<T>;
+  constexpr int N = VT::N, H2 = N / 2, EB = (int)sizeof(T);
+  uint32_t row[J], g[J];
+  bool isk[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const uint32_t w = it[j * stride];
+    row[j] = st + (w & kItemOffMask);
+    isk[j] = ((w >> kItemKindShift) & 3) != 0;
+    g[j] = isk[j] ? gk : gq;
+  }
+  float2 xa[J][H2], xb[J][H2];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    float t[N];
+    VT::widen(lds_v4(row[j] + cl.ca * EB), t);
+#pragma unroll
+    for (int k = 0; k < H2; ++k) xa[j][k] = make_float2(t[2 * k], t[2 * k + 1]);
+    VT::widen(lds_v4(row[j] + cl.cb * EB), t);
+#pragma unroll
+    for (int k = 0; k < H2; ++k) xb[j][k] = make_float2(t[2 * k], t[2 * k + 1]);
+  }
+  float r[J];
+  if constexpr (NORM) {
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      float2 acc = __fmul2_rn(xa[j][0], xa[j][0]);
+      acc = __ffma2_rn(xb[j][0], xb[j][0], acc);
+#pragma unroll
+      for (int k = 1; k < H2; ++k) {
+        acc = __ffma2_rn(xa[j][k], xa[j][k], acc);
+        acc = __ffma2_rn(xb[j][k], xb[j][k], acc);
+      }
+      r[j] = acc.x + acc.y;
+    }
+#pragma unroll
+    for (int msk = L / 2; msk > 0; msk >>= 1)
+#pragma unroll
+      for (int j = 0; j < J; ++j) r[j] += __shfl_xor_sync(cl.gmask, r[j], msk);
+    float ga_[N], gb_[N];  // gamma + weight_offset of the lane's columns, read once per kind
+    float(&ga)[N] = KG ? lg.a : ga_;
+    float(&gb)[N] = KG ? lg.b : gb_;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      r[j] = rsqrtf(r[j] * (1.0f / D) + eps);
+      if (KG ? g[j] != lg.addr : (j == 0 || g[j] != g[j - 1])) {
+        lds_f32<N>(g[j] + cl.ca * 4, cl.li, ga);
+        lds_f32<N>(g[j] + cl.cb * 4, cl.li, gb);
+        if (KG) lg.addr = g[j];
+      }
+      if (mbc) {  // x * gamma now; the scalar r after the rotation
+#pragma unroll
+        for (int k = 0; k < H2; ++k) {
+          xa[j][k] = __fmul2_rn(xa[j][k], make_float2(ga[2 * k], ga[2 * k + 1]));
+          xb[j][k] = __fmul2_rn(xb[j][k], make_float2(gb[2 * k], gb[2 * k + 1]));
+        }
+      } else {  // the normalised value is rounded to the element type, then scaled
+        const float2 rr = make_float2(r[j], r[j]);
+#pragma unroll
+        for (int k = 0; k < H2; ++k) {
+          xa[j][k] = __fmul2_rn(round2<T>(__fmul2_rn(xa[j][k], rr)),
+                                make_float2(ga[2 * k], ga[2 * k + 1]));
+          xb[j][k] = __fmul2_rn(round2<T>(__fmul2_rn(xb[j][k], rr)),
+                                make_float2(gb[2 * k], gb[2 * k + 1]));
+        }
+        r[j] = 1.f;
+      }
+    }
+    if constexpr (!EF) load_lane_freqs<N, INTER>(fr, cl, F);
+  }
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    rotate_lane<H2, INTER>(fr, cl, xa[j], xb[j]);
+    if constexpr (NORM) {
+      const float2 rr = make_float2(r[j], r[j]);
+#pragma unroll
+      for (int k = 0; k < H2; ++k) {
+        xa[j][k] = __fmul2_rn(xa[j][k], rr);
+        xb[j][k] = __fmul2_rn(xb[j][k], rr);
+      }
+    }
+    float ta[N], tb[N];
+#pragma unroll
+    for (int k = 0; k < H2; ++k) {
+      ta[2 * k] = xa[j][k].x;
+      ta[2 * k + 1] = xa[j][k].y;
+      tb[2 * k] = xb[j][k].x;
+      tb[2 * k + 1] = xb[j][k].y;
+    }
+    if constexpr (EXT) {
+      const int rb = (int)(row[j] - bo.blk) / (D * EB);  // the row's index in the band block
+      if (!isk[j] && bo.q_conv) {  // every lane writes its Q vectors, rounded once
+        const uint32_t qrow = bo.qo + (uint32_t)(rb * D * bo.q_eb);
+        sts_elems<N>(qrow + cl.ca * bo.q_eb, ta, bo.q_dtype);
+        sts_elems<N>(qrow + cl.cb * bo.q_eb, tb, bo.q_dtype);
+        continue;
+      }
+      if (isk[j] && bo.kv8) {  // and its K codes
+#pragma unroll
+        for (int e = 0; e < N; ++e) {
+          ta[e] *= bo.kinv;
+          tb[e] *= bo.kinv;
+        }
+        const uint32_t krow = bo.k8 + (uint32_t)((rb - bo.n_q) * D);
+        sts_e4m3<N>(krow + cl.ca, ta);
+        sts_e4m3<N>(krow + cl.cb, tb);
+        continue;
+      }
+    }
+    if (NORM || cl.rot_a) sts_v4(row[j] + cl.ca * EB, VT::narrow(ta));
+    if (NORM || cl.rot_b) sts_v4(row[j] + cl.cb * EB, VT::narrow(tb));
+  }
+}
+
+// A band's slots [lo, hi) of a consumer thread's head rows, JM at a time.  Without the norm
+// (and, if so built, one row at a time) the table row is read once here, for every chunk.
+#ifndef ROPE_ONE_ROW_EARLY_FREQS
+#define ROPE_ONE_ROW_EARLY_FREQS 1
+#endif
+#ifndef ROPE_ONE_ROW_KEEP_GAMMA
+#define ROPE_ONE_ROW_KEEP_GAMMA 0
+#endif
+template <int JM, typename T, int D, bool NORM, int L, bool INTER, bool EXT>
+__device__ __forceinline__ void rows_band(const ConsumerLane &cl, const uint32_t *item, int stride,
+                                          int lo, int hi, uint32_t st, uint32_t gq, uint32_t gk,
+                                          float eps, int mbc, const unsigned char *F,
+                                          LaneGamma<Vec<T>::N> &lg, const BandOut &bo) {
+  // one row at a time: the table row once per band and token, gamma kept across rows
+  constexpr bool EF = !NORM || (JM == 1 && ROPE_ONE_ROW_EARLY_FREQS);
+  constexpr bool KG = NORM && JM == 1 && ROPE_ONE_ROW_KEEP_GAMMA;
+  LaneFreqs<Vec<T>::N, INTER> fr;
+  if constexpr (EF) load_lane_freqs<Vec<T>::N, INTER>(fr, cl, F);
+  int u = lo;
+#pragma unroll 1
+  for (; u + JM <= hi; u += JM)
+    rows_step<JM, T, D, NORM, L, INTER, EXT, EF, KG>(cl, item + u * stride, stride, st, gq, gk,
+                                                    eps, mbc, F, fr, lg, bo);
+  if constexpr (JM >= 3) {
+    if (hi - u == 2)
+      rows_step<2, T, D, NORM, L, INTER, EXT, EF, KG>(cl, item + u * stride, stride, st, gq, gk,
+                                                     eps, mbc, F, fr, lg, bo);
+  }
+  if constexpr (JM >= 2) {
+    if (hi - u == 1)
+      rows_step<1, T, D, NORM, L, INTER, EXT, EF, KG>(cl, item + u * stride, stride, st, gq, gk,
+                                                     eps, mbc, F, fr, lg, bo);
+  }
+}
+
+#ifndef ROPE_LIGHT_MIN_CTAS
+#define ROPE_LIGHT_MIN_CTAS 3
+#endif
+// resident CTAs per SM the register budget is sized for: the light store shape (<= 4
+// consumer warps, no norm) and every other one
+template <int CW, bool NORM>
+__host__ __device__ constexpr int pipe_min_ctas() {
+  return CW <= 4 && !NORM ? ROPE_LIGHT_MIN_CTAS : 2;
+}
 
 // EXT: built with the extended outputs (a Q output in another element type, FP8 cache rows)
 template <typename T, int D, bool NORM, int CW, int LAG, bool EXT>
-__global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
+__global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
     banded_store_kernel(const __grid_constant__ BandedParams p) {
   constexpr int kConsumerWarps = CW;
   constexpr int kConsumers = 32 * CW;
@@ -353,7 +767,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         mj.stop = 0;
         const int s = issued % p.S;
         if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
+          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
             aborted = true;
           } else {
             meta[s] = mj;
@@ -425,7 +839,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     // stop marker: the next stage carries no token
     if (!aborted && lane == 0) {
       const int s = issued % p.S;
-      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
+      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
         aborted = true;
       } else {
         meta[s].stop = 1;
@@ -444,16 +858,81 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------------- storer --
-    if (lane == 0) {
+    // With an FP8 cache that takes V, every lane of the warp first encodes the staged V rows
+    // (nothing else reads them): E4M3 codes of value / scale, each rounded exactly once.
+    const bool venc = EXT && ((p.band[0].kv8 && p.band[0].n_v) ||
+                              (p.n_bands > 1 && p.band[1].kv8 && p.band[1].n_v));
+    if (lane == 0 || venc) {
       int n_done = 0;  // tokens stored
+      float vs[2] = {1.f, 1.f}, vinv[2] = {1.f, 1.f};
       for (int i = 0;; ++i) {
         const int s = i % p.S;
-        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort)) {
-          s_abort = 1;
-          raise(p.err, ROPE_DEVERR_TIMEOUT);
-          break;
+        if constexpr (EXT) {
+          if (venc) {
+            const bool got =
+                __all_sync(0xffffffffu, mbar_wait(&full[s], (i / p.S) & 1, &s_abort, p.wait_polls));
+            if (!got) {
+              if (lane == 0) {
+                s_abort = 1;
+                raise(p.err, ROPE_DEVERR_TIMEOUT);
+              }
+              break;
+            }
+            if (i == 0) {  // after the producer's wait for the preceding kernels
+#pragma unroll
+              for (int k = 0; k < 2; ++k)
+                if (k < p.n_bands && (k ? p.band[1] : p.band[0]).kv8 &&
+                    (k ? p.band[1] : p.band[0]).n_v) {
+                  vs[k] = __ldg((k ? p.band[1] : p.band[0]).v_scale);
+                  vinv[k] = 1.f / vs[k];
+                }
+            }
+            if (!meta[s].stop) {
+              const uint32_t st = smem_addr(stages) + (uint32_t)(s * p.stage_bytes);
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {
+                if (k >= p.n_bands || !meta[s].ok[k]) continue;
+                const BandDev &bd = k ? p.band[1] : p.band[0];
+                if (!bd.kv8 || !bd.n_v) continue;
+                const uint32_t vblk = st + (uint32_t)(bd.smem_off + (bd.n_q + bd.n_kv) * D * EB);
+                const uint32_t v8 = st + (uint32_t)bd.v8_off;
+                const int nvec = bd.n_v * D / N;
+                for (int vv = lane; vv < nvec; vv += 32) {
+                  float x[N];
+                  VT::widen(lds_v4(vblk + vv * 16), x);
+                  uint32_t w[N / 4];
+#pragma unroll
+                  for (int q = 0; q < N / 4; ++q)
+                    w[q] = e4m3_exact4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3],
+                                       vinv[k], vs[k]);
+                  if constexpr (N == 8) {
+                    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(v8 + vv * N),
+                                 "r"(w[0]), "r"(w[N / 4 - 1])
+                                 : "memory");
+                  } else {
+                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(v8 + vv * N), "r"(w[0])
+                                 : "memory");
+                  }
+                }
+              }
+              fence_proxy_async_smem();  // the bulk copies below read these codes
+            }
+            __syncwarp();
+          }
         }
-        if (meta[s].stop) break;
+        int stop = 0;
+        if (lane == 0) {
+          if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
+            s_abort = 1;
+            raise(p.err, ROPE_DEVERR_TIMEOUT);
+            stop = 2;
+          } else if (meta[s].stop) {
+            stop = 1;
+          }
+        }
+        if (venc) stop = __shfl_sync(0xffffffffu, stop, 0);
+        if (stop) break;
+        if (lane != 0) continue;
         n_done = i + 1;
         const uint32_t tok = (uint32_t)meta[s].tok;
         const unsigned char *st = stages + (size_t)s * p.stage_bytes;
@@ -498,16 +977,21 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
           mbar_arrive(&empty[(i - kStoreLag) % p.S]);
         }
       }
-      bulk_wait_read<0>();
-      for (int i = max(0, n_done - kStoreLag); i < n_done; ++i) mbar_arrive(&empty[i % p.S]);
-      bulk_wait<0>();
+      if (lane == 0) {
+        bulk_wait_read<0>();
+        for (int i = max(0, n_done - kStoreLag); i < n_done; ++i) mbar_arrive(&empty[i % p.S]);
+        bulk_wait<0>();
+      }
     }
   } else {
     // ------------------------------------------------------------------ consumers --
     // A head row is D / N 16-byte vectors; lane j of its group of L lanes owns two of them,
     // va and vb.  Half-split: the first R/(2N) lanes own a rotation pair each (vector
     // o/N + j and its partner R/(2N) vectors later), the other lanes own two unrotated
-    // vectors.  Interleaved: lane j owns vectors j and j + L.
+    // vectors.  Interleaved: lane j owns vectors j and j + L.  A thread's head rows of a
+    // token are taken up to JM at a time, so that their load -> reduce -> scale -> rotate
+    // chains overlap.
+    constexpr int JM = chunk_rows<CW, NORM>();
     const int ctid = tid - 64;
     const int li = ctid % L, grp = ctid / L;
     const unsigned gmask = (L == 32) ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
@@ -535,13 +1019,14 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
     }
     const bool busy = NORM || rot_a || rot_b;  // lanes with nothing to do leave bytes in place
     const int ca = va * N, cb = vb * N;         // first columns of the two vectors
-    // table columns: interleaved, vector v uses F[v*N - off ..]; half-split pair uses
-    // F[2 * (ca - off) ..] (cos, sin of pair ca - off + e)
     const int fa = inter ? ca - rp.off : 2 * (ca - rp.off);
     const int fb = cb - rp.off;
-    // this thread's head rows of a token, decoded once into shared memory
+    const ConsumerLane cl{li, ca, cb, fa, fb, rp.dtype, inter, rot_a, rot_b, gmask};
+    // this thread's head rows of a token, decoded once into shared memory: rows of band 0
+    // in slots [0, u_end0), of band 1 in [u_end0, u_end1)
     const int n_items = (p.work_total + G - 1) / G;
     uint32_t *item = s_items + ctid;  // slot u at item[u * kConsumers]
+    int u_end0 = 0, u_end1 = 0;
     for (int u = 0; u < n_items; ++u) {
       const int j = grp + u * G;
       uint32_t w = 0;
@@ -549,20 +1034,22 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         const int band = j >= p.work0 ? 1 : 0;
         const BandDev &bd = band ? p.band[1] : p.band[0];
         const int r = j - (band ? p.work0 : 0);  // Q heads then K heads: stage rows 0..
-        const int kind = r < bd.n_q ? 0 : r < bd.n_q + bd.n_kv ? 1 : 2;
+        const int kind = r < bd.n_q ? 0 : 1;
         const uint32_t soff = (uint32_t)(bd.smem_off + r * D * EB);
         w = kItemAct | (uint32_t)band << kItemBandShift | (uint32_t)kind << kItemKindShift | soff;
+        if (band == 0) u_end0 = u + 1;
+        u_end1 = u + 1;
       }
       item[u * kConsumers] = w;
     }
-    // per token: (cos, sin) of this lane's columns; per (band, kind): gamma + weight_offset
-    float fca[N], fsa[N], fcb[N], fsb[N];
-    float ga[N], gb[N];
-    int g_sel = -1;
-    float kinv0 = 1.f, kinv1 = 1.f, vinv0 = 1.f, vinv1 = 1.f;  // 1 / scale of FP8 planes
+    const uint32_t stages_a = smem_addr(stages);
+    const uint32_t gamma_a = smem_addr(s_gamma);
+    float kinv[2] = {1.f, 1.f};  // 1 / scale of FP8 K planes
+    LaneGamma<N> lg;             // one-row chunks: the gamma last read, kept across rows
+    lg.addr = ~0u;
     for (int i = 0;; ++i) {
       const int s = i % p.S;
-      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
+      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
         if (lane == 0) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);
@@ -575,168 +1062,33 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW>())
         break;
       }
       if (EXT && i == 0) {  // after the producer's wait for the preceding kernels
-        if (p.band[0].kv8) {
-          kinv0 = 1.f / __ldg(p.band[0].k_scale);
-          if (p.band[0].n_v) vinv0 = 1.f / __ldg(p.band[0].v_scale);
-        }
-        if (p.n_bands > 1 && p.band[1].kv8) {
-          kinv1 = 1.f / __ldg(p.band[1].k_scale);
-          if (p.band[1].n_v) vinv1 = 1.f / __ldg(p.band[1].v_scale);
-        }
+        if (p.band[0].kv8) kinv[0] = 1.f / __ldg(p.band[0].k_scale);
+        if (p.n_bands > 1 && p.band[1].kv8) kinv[1] = 1.f / __ldg(p.band[1].k_scale);
       }
-      unsigned char *st = stages + (size_t)s * p.stage_bytes;
+      const uint32_t st = stages_a + (uint32_t)(s * p.stage_bytes);
       const int ok0 = meta[s].ok[0], ok1 = meta[s].ok[1];
-      int f_band = -1;
 #pragma unroll 1
-      for (int u = 0; u < n_items; ++u) {
-        const uint32_t w = item[u * kConsumers];
-        if (!(w & kItemAct)) continue;
-        const int band = (w >> kItemBandShift) & 1;
-        if (!(band ? ok1 : ok0)) continue;
-        const int kind = (w >> kItemKindShift) & 3;
+      for (int band = 0; band < p.n_bands; ++band) {
+        const int lo = band ? u_end0 : 0, hi = band ? u_end1 : u_end0;
+        if (lo >= hi || !(band ? ok1 : ok0)) continue;
         const BandDev &bd = band ? p.band[1] : p.band[0];
-        const bool conv = EXT && kind == 0 && bd.q_conv;  // every lane writes its Q
-        const bool to8 = EXT && kind >= 1 && bd.kv8;       // and its K / V codes
-        if (!busy && !conv && !to8) continue;
-        if ((rot_a || rot_b) && f_band != band) {  // this token's table row for the band
-          f_band = band;
-          const unsigned char *F = st + bd.f_off;
-          if (inter) {
-            float f[N];
-            if (rot_a) {
-              lds_freqs<N>(F, rp.dtype, fa, li, f);
-#pragma unroll
-              for (int e = 0; e < N; e += 2) {
-                fca[e] = fca[e + 1] = f[e];
-                fsa[e] = fsa[e + 1] = f[e + 1];
-              }
-            }
-            if (rot_b) {
-              lds_freqs<N>(F, rp.dtype, fb, li, f);
-#pragma unroll
-              for (int e = 0; e < N; e += 2) {
-                fcb[e] = fcb[e + 1] = f[e];
-                fsb[e] = fsb[e + 1] = f[e + 1];
-              }
-            }
-          } else {
-            float f[2 * N];
-            lds_freqs<2 * N>(F, rp.dtype, fa, li, f);
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-              fca[e] = f[2 * e];
-              fsa[e] = f[2 * e + 1];
-            }
-          }
+        // lanes with nothing to do leave their bytes in place, unless they go elsewhere
+        if (!busy && !(EXT && (bd.q_conv || bd.kv8))) continue;
+        const unsigned char *F = stages + (size_t)s * p.stage_bytes + bd.f_off;
+        const float eps = bd.eps;
+        const uint32_t gq = gamma_a + (uint32_t)(band * 2 * D * 4), gk = gq + D * 4;
+        BandOut bo{};
+        if constexpr (EXT) {
+          bo = BandOut{st + (uint32_t)bd.smem_off, st + (uint32_t)bd.qo_off,
+                       st + (uint32_t)bd.k8_off, bd.q_conv, bd.q_dtype, bd.q_eb, bd.kv8, bd.n_q,
+                       kinv[band]};
         }
-        unsigned char *row = st + (w & kItemOffMask);
-        float xa[N], xb[N];
-        VT::widen(ld_shared_v4(row + ca * EB), xa);
-        VT::widen(ld_shared_v4(row + cb * EB), xb);
-        // the row's first element within the band's [Q | K | V] block
-        const int re = (int)(((w & kItemOffMask) - (uint32_t)bd.smem_off) / EB);
-        if (EXT && kind == 2) {  // a V row of an FP8 cache: scaled and encoded, nothing else
-          const float inv = band ? vinv1 : vinv0;
-#pragma unroll
-          for (int e = 0; e < N; ++e) {
-            xa[e] *= inv;
-            xb[e] *= inv;
-          }
-          unsigned char *vrow = st + bd.v8_off + (re - (bd.n_q + bd.n_kv) * D);
-          st_shared_e4m3<N>(vrow + ca, xa);
-          st_shared_e4m3<N>(vrow + cb, xb);
-          continue;
-        }
-        if constexpr (NORM) {
-          if (g_sel != band * 2 + kind) {  // gamma does not depend on the token: kept
-            g_sel = band * 2 + kind;
-            const unsigned char *gr = reinterpret_cast<const unsigned char *>(s_gamma + g_sel * D);
-            lds_freqs<N>(gr, 2, ca, li, ga);
-            lds_freqs<N>(gr, 2, cb, li, gb);
-          }
-          float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int e = 0; e < N; e += 2) {
-            acc = __ffma2_rn(make_float2(xa[e], xa[e + 1]), make_float2(xa[e], xa[e + 1]), acc);
-            acc = __ffma2_rn(make_float2(xb[e], xb[e + 1]), make_float2(xb[e], xb[e + 1]), acc);
-          }
-          float ss = acc.x + acc.y;
-#pragma unroll
-          for (int msk = L / 2; msk > 0; msk >>= 1) ss += __shfl_xor_sync(gmask, ss, msk);
-          const float r = rsqrtf(ss * (1.0f / D) + bd.eps);
-          const float2 rr = make_float2(r, r);
-          if (p.mbc) {
-#pragma unroll
-            for (int e = 0; e < N; e += 2) {
-              const float2 ya = __fmul2_rn(make_float2(xa[e], xa[e + 1]),
-                                           __fmul2_rn(rr, make_float2(ga[e], ga[e + 1])));
-              const float2 yb = __fmul2_rn(make_float2(xb[e], xb[e + 1]),
-                                           __fmul2_rn(rr, make_float2(gb[e], gb[e + 1])));
-              xa[e] = ya.x; xa[e + 1] = ya.y;
-              xb[e] = yb.x; xb[e + 1] = yb.y;
-            }
-          } else {  // the normalised value is rounded to the element type, then scaled
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-              xa[e] *= r;
-              xb[e] *= r;
-            }
-            VT::widen(VT::narrow(xa), xa);
-            VT::widen(VT::narrow(xb), xb);
-#pragma unroll
-            for (int e = 0; e < N; ++e) {
-              xa[e] *= ga[e];
-              xb[e] *= gb[e];
-            }
-          }
-        }
-        if (inter) {
-          if (rot_a) {
-#pragma unroll
-            for (int e = 0; e < N; e += 2) {
-              const float a = xa[e], b = xa[e + 1];
-              xa[e] = fmaf(a, fca[e], -b * fsa[e]);
-              xa[e + 1] = fmaf(a, fsa[e], b * fca[e]);
-            }
-          }
-          if (rot_b) {
-#pragma unroll
-            for (int e = 0; e < N; e += 2) {
-              const float a = xb[e], b = xb[e + 1];
-              xb[e] = fmaf(a, fcb[e], -b * fsb[e]);
-              xb[e + 1] = fmaf(a, fsb[e], b * fcb[e]);
-            }
-          }
-        } else if (rot_a) {
-          // (a, b) -> (a c - b s, a s + b c), pair e of vector va with pair e of vector vb
-#pragma unroll
-          for (int e = 0; e < N; e += 2) {
-            const float2 a = make_float2(xa[e], xa[e + 1]), b = make_float2(xb[e], xb[e + 1]);
-            const float2 c = make_float2(fca[e], fca[e + 1]), sn = make_float2(fsa[e], fsa[e + 1]);
-            const float2 ya = __ffma2_rn(b, make_float2(-sn.x, -sn.y), __fmul2_rn(a, c));
-            const float2 yb = __ffma2_rn(a, sn, __fmul2_rn(b, c));
-            xa[e] = ya.x; xa[e + 1] = ya.y;
-            xb[e] = yb.x; xb[e + 1] = yb.y;
-          }
-        }
-        if (conv) {
-          unsigned char *qrow = st + bd.qo_off + (size_t)re * bd.q_eb;
-          st_shared_elems<N>(qrow + ca * bd.q_eb, xa, bd.q_dtype);
-          st_shared_elems<N>(qrow + cb * bd.q_eb, xb, bd.q_dtype);
-        } else if (to8) {  // a K row of an FP8 cache
-          const float inv = band ? kinv1 : kinv0;
-#pragma unroll
-          for (int e = 0; e < N; ++e) {
-            xa[e] *= inv;
-            xb[e] *= inv;
-          }
-          unsigned char *krow = st + bd.k8_off + (re - bd.n_q * D);
-          st_shared_e4m3<N>(krow + ca, xa);
-          st_shared_e4m3<N>(krow + cb, xb);
-        } else {
-          if (NORM || rot_a) st_shared_v4(row + ca * EB, VT::narrow(xa));
-          if (NORM || rot_b) st_shared_v4(row + cb * EB, VT::narrow(xb));
-        }
+        if (inter)
+          rows_band<JM, T, D, NORM, L, true, EXT>(cl, item, kConsumers, lo, hi, st, gq, gk, eps,
+                                                 p.mbc, F, lg, bo);
+        else
+          rows_band<JM, T, D, NORM, L, false, EXT>(cl, item, kConsumers, lo, hi, st, gq, gk,
+                                                  eps, p.mbc, F, lg, bo);
       }
       fence_proxy_async_smem();  // the storer's bulk copies read what was written here
       __syncwarp();

@@ -32,6 +32,7 @@ struct GemvParams {
   uint32_t *err;
   int32_t overlap;
   int32_t row_bytes;  // k * element size, padded to 16: a row's place in shared memory
+  uint32_t wait_polls;  // the most polls of the load wait (the drain keeps kSpinLimit)
 };
 
 template <typename T>
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(kGemvThreads)
                  kb, &bar);
     }
     bool ok = true;
-    if (kb > 0 && !mbar_wait(&bar, 0, &s_abort)) {
+    if (kb > 0 && !mbar_wait(&bar, 0, &s_abort, p.wait_polls)) {
       ok = false;
       if (lane == 0) raise(p.err, ROPE_DEVERR_TIMEOUT);
     }

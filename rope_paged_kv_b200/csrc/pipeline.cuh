@@ -62,14 +62,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
+// The same test without the hardware's suspend: returns at once.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up (returns
-// false) after kWaitLimitNs of wall time or kSpinLimit polls, or early once *abort is set
-// by another thread of the CTA.
+// false) after kWaitLimitNs of wall time or max_polls polls (kSpinLimit unless a caller
+// asks for fewer), or early once *abort is set by another thread of the CTA.  A caller's
+// smaller poll limit polls without the hardware's suspend (mbarrier.try_wait may sleep a
+// while before it fails), so that such a wait runs out after max_polls quick tests.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          const volatile int *abort) {
+                                          const volatile int *abort,
+                                          uint32_t max_polls = kSpinLimit) {
   uint64_t t0 = 0;
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+  const bool quick = max_polls < kSpinLimit;
+  for (uint32_t it = 0; it < max_polls; ++it) {
+    if (quick ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
 #if ROPE_WAIT_BACKOFF_NS > 0
     if (it >= 2) __nanosleep(ROPE_WAIT_BACKOFF_NS);  // leave the issue slots to busy warps
 #endif
@@ -149,6 +166,20 @@ __device__ __forceinline__ uint4 ld_shared_v4(const void *p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(smem_addr(p)));
   return v;
+}
+
+// the same with 32-bit shared-memory addresses
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_v4(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 }  // namespace rs

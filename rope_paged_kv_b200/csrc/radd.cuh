@@ -25,6 +25,7 @@ struct RaddParams {
   int32_t S, stage_bytes, staged, kv_contig;  // kv_contig: a token's heads are adjacent
   int32_t bar_off, meta_off, offs_off;
   int32_t overlap;  // launch-overlap mode (kOverlap*)
+  uint32_t wait_polls;  // the most polls of a pipeline wait (drains keep kSpinLimit)
   uint32_t *sched;  // claim counter + finished CTAs, or nullptr for a static schedule
 };
 
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
         mj.tok = __shfl_sync(0xffffffffu, m.tok, j);
         const int s = issued % p.S;
         if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
+          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
             aborted = true;
           } else {
             meta[s] = mj;
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
     }
     if (!aborted && lane == 0) {  // stop marker
       const int s = issued % p.S;
-      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
+      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
         aborted = true;
       } else {
         meta[s].stop = 1;
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
       int n_done = 0;
       for (int i = 0;; ++i) {
         const int s = i % p.S;
-        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort)) {
+        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);
           break;
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
     const int rows = 2 * p.n_kv;
     for (int i = 0;; ++i) {
       const int s = i % p.S;
-      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
+      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
         if (lane == 0) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);

@@ -43,8 +43,18 @@ constexpr BandedShape kLightShape = {ROPE_LIGHT_CW, ROPE_LIGHT_LAG, ROPE_LIGHT_R
 // token's head rows (six on a tie: 116.6 vs 119.9 us on the per-head-norm workload, whose
 // 72 rows take three passes either way; eight on the dual-band one, 81 rows in three
 // passes instead of four: 248.4 vs 264.8 us)
-constexpr BandedShape kMidShape = {6, 0, 96};
-constexpr BandedShape kHeavyShape = {8, 0, 96};
+#ifndef ROPE_MID_CW
+#define ROPE_MID_CW 6
+#define ROPE_MID_LAG 0
+#define ROPE_MID_RING 96
+#endif
+#ifndef ROPE_HEAVY_CW
+#define ROPE_HEAVY_CW 8
+#define ROPE_HEAVY_LAG 0
+#define ROPE_HEAVY_RING 96
+#endif
+constexpr BandedShape kMidShape = {ROPE_MID_CW, ROPE_MID_LAG, ROPE_MID_RING};
+constexpr BandedShape kHeavyShape = {ROPE_HEAVY_CW, ROPE_HEAVY_LAG, ROPE_HEAVY_RING};
 
 enum ShapeId { kLight = 0, kMid = 1, kHeavy = 2 };
 
@@ -54,12 +64,12 @@ static int passes(const BandedParams &p, int D, int cw) {
 }
 
 static ShapeId pick_shape(const BandedParams &p, int D, bool norm) {
-  // an FP8 cache without norm: six consumer warps, since its V rows pass through the
-  // consumers too (Llama-3-8B prefill into an FP8 cache: 52.8 us, 59.7 in the light shape,
-  // 55.5 in the heavy one)
-  if (!norm && p.band[0].kv8) return kMid;
-  // few head rows without norm, or Q converted to another type: the light shape
+  // few head rows without norm, or Q converted to another type: the light shape (the V rows
+  // of an FP8 cache are encoded by the storer warp, not by the consumers)
   if (!norm && (p.work_total <= 64 || p.band[0].q_conv)) return kLight;
+#ifdef ROPE_NORM_ALWAYS_MID
+  if (norm) return kMid;
+#endif
   return passes(p, D, kMidShape.cw) <= passes(p, D, kHeavyShape.cw) ? kMid : kHeavy;
 }
 
@@ -71,6 +81,13 @@ static const BandedShape &shape_of(ShapeId id) {
 
 // launch-overlap mode of every launch that follows (rope_set_launch_overlap)
 static std::atomic<int> g_overlap{kOverlapPdl};
+// the most polls of a pipeline wait in the launches that follow (rope_set_wait_limit; 0: the
+// default)
+static std::atomic<uint32_t> g_wait_polls{0};
+static uint32_t wait_polls() {
+  const uint32_t w = g_wait_polls.load(std::memory_order_relaxed);
+  return w ? w : kSpinLimit;
+}
 
 // Launch `kern` with one parameter block; modes 1 and 2 launch it as a programmatic
 // dependent of the previous kernel in the stream.
@@ -364,9 +381,12 @@ static rope_status_t launch_banded_s(ShapeId id, const BandedParams &p, size_t s
                                      cudaStream_t st) {
   // Q in another element type or an FP8 cache: the instantiation with those outputs
   const bool ext = p.band[0].q_conv || p.band[0].kv8 || (p.n_bands > 1 && p.band[1].kv8);
-  if (id == kLight)
-    return ext ? launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag, true>(p, smem, st)
-               : launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
+  if constexpr (!NORM) {  // (the light shape is never picked for a launch with the norm)
+    if (id == kLight)
+      return ext ? launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag, true>(p, smem,
+                                                                                      st)
+                 : launch_banded_t<T, D, NORM, kLightShape.cw, kLightShape.lag>(p, smem, st);
+  }
   if (id == kMid)
     return ext ? launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag, true>(p, smem, st)
                : launch_banded_t<T, D, NORM, kMidShape.cw, kMidShape.lag>(p, smem, st);
@@ -505,6 +525,46 @@ static rope_status_t launch_gemv_t(const GemvParams &p, cudaStream_t st) {
   return launch_gemv_r<T, 8>(p, st);
 }
 
+// Argument checks and parameter block of rope_split_store_paged_ragged (total_tokens > 0);
+// *work is false when the call has nothing to launch.  Nothing is queued on any stream.
+static rope_status_t prepare_ragged_store(const void *qkv, int64_t qkv_row_stride,
+                                          int32_t qkv_dtype, int32_t total_tokens,
+                                          int32_t n_q_heads, const uint32_t *input_row_offsets,
+                                          int32_t batch, const rope_freqs_t *freqs,
+                                          const rope_paged_cache_t *kv, uint32_t layer_idx,
+                                          void *q_out, int64_t q_out_row_stride,
+                                          int32_t q_out_dtype, uint32_t *err_word,
+                                          uint32_t *sched, BandedParams &p, int &dtype, int &D,
+                                          bool &work) {
+  work = false;
+  if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
+  // the input's element type: given, or the cache's
+  dtype = qkv_dtype >= 0 ? qkv_dtype : kv->dtype;
+  D = kv->head_dim;
+  rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
+  if (s != ROPE_OK) return s;
+  if (batch > kv->n_seqs || n_q_heads < 0) return ROPE_ERR_INVALID_ARG;
+  s = check_freqs(freqs, dtype, D, &p.rope);
+  if (s != ROPE_OK) return s;
+  const int64_t Hq = n_q_heads, Hk = kv->n_kv_heads;
+  s = fill_band(&p.band[0], qkv, qkv_row_stride, 0, Hq * D, (Hq + Hk) * D, n_q_heads, kv,
+                nullptr, nullptr, 0.f, q_out, q_out_row_stride, dtype, layer_idx, false,
+                q_out_dtype);
+  if (s != ROPE_OK) return s;
+  p.n_bands = 1;
+  p.work0 = p.work_total = (int32_t)(Hq + Hk);  // the head rows the consumers take: Q and K
+  p.offs = input_row_offsets;
+  p.batch = batch;
+  p.T = total_tokens;
+  p.layer = layer_idx;
+  p.err = err_word;
+  p.sched = sched;
+  p.overlap = g_overlap.load(std::memory_order_relaxed);
+  p.wait_polls = wait_polls();
+  work = p.work_total + Hk > 0;  // V alone (no Q or K heads) is still copied
+  return ROPE_OK;
+}
+
 // ------------------------------------------------------- allocation-free entry point --
 // Scheduling workspace of rope_split_store_paged_ragged_noalloc.  Every device that loads
 // the library holds one copy of this array until the process exits, and every call of that
@@ -514,21 +574,54 @@ constexpr int kNoAllocScratchWords = 64;  // 256 bytes
 static_assert(ROPE_SCHED_WORDS <= kNoAllocScratchWords, "the schedule must fit the array");
 static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocScratchWords];
 
-// The array's device address on the current device.  In host code the symbol only names a
-// host-side stand-in, so the address is looked up once per device, with that device
-// current, and cached; nullptr if the lookup fails.
+// Identity of the calling thread's current CUDA context: its process-unique id (the driver's
+// cuCtxGetId, reached through the runtime without linking the driver library), or 0 when no
+// context is current or the driver cannot tell.
+typedef int (*CtxGetCurrentFn)(void **);
+typedef int (*CtxGetIdFn)(void *, unsigned long long *);
+static unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *a = nullptr, *b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 12000, cudaEnableDefault,
+                                         &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &qb) ==
+            cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+  });
+  void *ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_current(&ctx) != 0 || ctx == nullptr || get_id(ctx, &id) != 0)
+    return 0;
+  return id;
+}
+
+// The array's device address in the current device's context.  In host code the symbol only
+// names a host-side stand-in, so the address is looked up with cudaGetSymbolAddress (with the
+// device current) and kept, together with the id of the context it belongs to: a context
+// made after a device reset gets its own copy of the module, and with it a new lookup.
+// nullptr if the lookup fails.
 static uint32_t *noalloc_scratch() {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static uint32_t *addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = static_cast<uint32_t *>(p);
-  }
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0 && ctx == ctx_of[dev] && addr[dev] != nullptr) return addr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  addr[dev] = static_cast<uint32_t *>(p);
+  ctx_of[dev] = current_context_id();  // the lookup made the device's context current
   return addr[dev];
 }
 
@@ -558,31 +651,13 @@ rope_status_t rope_split_store_paged_ragged(const void *qkv, int64_t qkv_row_str
                                             int32_t q_out_dtype, uint32_t *err_word,
                                             uint32_t *sched, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
-  if (kv == nullptr || !sched_ok(sched)) return ROPE_ERR_INVALID_ARG;
-  // the input's element type: given, or the cache's
-  const int dtype = qkv_dtype >= 0 ? qkv_dtype : kv->dtype, D = kv->head_dim;
-  rope_status_t s = common_checks(dtype, D, input_row_offsets, batch, total_tokens);
-  if (s != ROPE_OK) return s;
-  if (batch > kv->n_seqs || n_q_heads < 0) return ROPE_ERR_INVALID_ARG;
   BandedParams p{};
-  s = check_freqs(freqs, dtype, D, &p.rope);
-  if (s != ROPE_OK) return s;
-  const int64_t Hq = n_q_heads, Hk = kv->n_kv_heads;
-  s = fill_band(&p.band[0], qkv, qkv_row_stride, 0, Hq * D, (Hq + Hk) * D, n_q_heads, kv,
-                nullptr, nullptr, 0.f, q_out, q_out_row_stride, dtype, layer_idx, false,
-                q_out_dtype);
-  if (s != ROPE_OK) return s;
-  p.n_bands = 1;
-  // head rows the consumers touch: Q and K, and V too when it is encoded for an FP8 cache
-  p.work0 = p.work_total = (int32_t)(Hq + Hk + (p.band[0].kv8 ? Hk : 0));
-  p.offs = input_row_offsets;
-  p.batch = batch;
-  p.T = total_tokens;
-  p.layer = layer_idx;
-  p.err = err_word;
-  p.sched = sched;
-  p.overlap = g_overlap.load(std::memory_order_relaxed);
-  if (p.work_total + Hk == 0) return ROPE_OK;
+  int dtype = 0, D = 0;
+  bool work = false;
+  const rope_status_t s = prepare_ragged_store(
+      qkv, qkv_row_stride, qkv_dtype, total_tokens, n_q_heads, input_row_offsets, batch, freqs,
+      kv, layer_idx, q_out, q_out_row_stride, q_out_dtype, err_word, sched, p, dtype, D, work);
+  if (s != ROPE_OK || !work) return s;
   return launch_banded(dtype, D, false, p, (cudaStream_t)stream);
 }
 
@@ -613,8 +688,7 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
                 q_gamma, k_gamma, epsilon, q_out, q_out_row_stride, dtype, layer_idx, true);
   if (s != ROPE_OK) return s;
   p.n_bands = 1;
-  // head rows the consumers touch: Q and K, and V too when it is encoded for an FP8 cache
-  p.work0 = p.work_total = (int32_t)(Hq + Hk + (p.band[0].kv8 ? Hk : 0));
+  p.work0 = p.work_total = (int32_t)(Hq + Hk);  // the head rows the consumers take: Q and K
   p.offs = input_row_offsets;
   p.batch = batch;
   p.T = total_tokens;
@@ -622,6 +696,7 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
+  p.wait_polls = wait_polls();
   p.weight_offset = round_to_elem(weight_offset, dtype);
   if (p.work_total + Hk == 0) return ROPE_OK;
   return launch_banded(dtype, D, true, p, (cudaStream_t)stream);
@@ -665,7 +740,7 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
                   b->n_q_heads, b->cache, b->q_gamma, b->k_gamma, b->epsilon, b->q_out,
                   b->q_out_row_stride, dtype, layer_idx, true);
     if (s != ROPE_OK) return s;
-    rows[k] = p.band[k].n_q + p.band[k].n_kv + (p.band[k].kv8 ? p.band[k].n_v : 0);
+    rows[k] = p.band[k].n_q + p.band[k].n_kv;  // the head rows the consumers take
   }
   p.n_bands = n_bands;
   p.work0 = rows[0];
@@ -677,6 +752,7 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
+  p.wait_polls = wait_polls();
   p.weight_offset = round_to_elem(weight_offset, dtype);
   if (p.work_total == 0) return ROPE_OK;
   return launch_banded(dtype, D, true, p, (cudaStream_t)stream);
@@ -759,6 +835,7 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
+  p.wait_polls = wait_polls();
   p.kv_contig = kv->head_stride == D ? 1 : 0;
   const size_t smem = layout_radd(p, D, eb);
   if (smem > 227 * 1024) return ROPE_ERR_UNSUPPORTED;
@@ -775,16 +852,23 @@ rope_status_t rope_split_store_paged_ragged_noalloc(
     const rope_paged_cache_t *kv, uint32_t layer_idx, void *q_out, int64_t q_out_row_stride,
     int32_t q_out_dtype, uint32_t *err_word, rope_stream_t stream) {
   if (total_tokens == 0) return ROPE_OK;  // no work: nothing is read or written
+  // every argument check first: a call that is rejected queues nothing on the stream
+  BandedParams p{};
+  int dtype = 0, D = 0;
+  bool work = false;
+  rope_status_t s = prepare_ragged_store(qkv, qkv_row_stride, qkv_dtype, total_tokens,
+                                         n_q_heads, input_row_offsets, batch, freqs, kv,
+                                         layer_idx, q_out, q_out_row_stride, q_out_dtype,
+                                         err_word, nullptr, p, dtype, D, work);
+  if (s != ROPE_OK || !work) return s;
   uint32_t *scratch = noalloc_scratch();
   if (scratch == nullptr) return ROPE_ERR_CUDA;
   // the workspace starts each call at zero (a call that gave up early may have left counts)
   if (cudaMemsetAsync(scratch, 0, ROPE_SCHED_WORDS * sizeof(uint32_t), (cudaStream_t)stream) !=
       cudaSuccess)
     return ROPE_ERR_CUDA;
-  return rope_split_store_paged_ragged(qkv, qkv_row_stride, qkv_dtype, total_tokens, n_q_heads,
-                                       input_row_offsets, batch, freqs, kv, layer_idx, q_out,
-                                       q_out_row_stride, q_out_dtype, err_word, scratch,
-                                       stream);
+  p.sched = scratch;
+  return launch_banded(dtype, D, false, p, (cudaStream_t)stream);
 }
 
 rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight,
@@ -827,6 +911,7 @@ rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight
   p.err = err_word;
   p.row_bytes = (int32_t)round_up((int64_t)k * eb, 16);
   p.overlap = g_overlap.load(std::memory_order_relaxed);
+  p.wait_polls = wait_polls();
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == ROPE_DTYPE_BF16) return launch_gemv_t<__nv_bfloat16>(p, st);
   if (dtype == ROPE_DTYPE_F16) return launch_gemv_t<__half>(p, st);
@@ -841,5 +926,12 @@ rope_status_t rope_set_launch_overlap(int32_t mode) {
 }
 
 int32_t rope_get_launch_overlap(void) { return g_overlap.load(std::memory_order_relaxed); }
+
+rope_status_t rope_set_wait_limit(uint32_t polls) {
+  g_wait_polls.store(polls, std::memory_order_relaxed);
+  return ROPE_OK;
+}
+
+uint32_t rope_get_wait_limit(void) { return g_wait_polls.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -4,11 +4,15 @@ Some callers cannot allocate device memory (an engine that owns the whole device
 latency-critical path that must not call cudaMalloc / cudaFree), so this entry point keeps
 its scheduling workspace in the library's own per-device array.  Called twice in a row
 through the C ABI, it must give what rope_split_store_paged_ragged gives with a caller-owned
-workspace, within the parity tolerance (rotated values) and bit for bit (everything else).
-This file is collected last, and it passes alone in a fresh process as well.
+workspace, within the parity tolerance (rotated values) and bit for bit (everything else),
+and match the oracle the same way.  It must allocate nothing: the device's free memory is
+the same before and after a run of calls.  A call that is rejected, or that has no tokens,
+queues nothing, and the next call is still right.  This file is collected last, and it
+passes alone in a fresh process as well.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
@@ -26,12 +30,44 @@ def _workload(seed):
                           interleaved=False, max_seq_len=4096)
 
 
-def test_noalloc_store_matches_the_store_with_a_workspace():
+@pytest.fixture(scope="module")
+def G():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    import gpu_helpers as G
-    import rope_paged_kv_b200 as rs
+    import gpu_helpers
+    return gpu_helpers
 
+
+def _noalloc(lib, w, s, stream, total_tokens=None, kv=None):
+    f = s.freqs.c()
+    c = s.kv.c() if kv is None else kv
+    return lib.rope_split_store_paged_ragged_noalloc(
+        s.qkv.data_ptr(), s.qkv.stride(0), -1,
+        w.total_tokens if total_tokens is None else total_tokens, w.n_q_heads,
+        s.offs.data_ptr(), s.offs.shape[0] - 1, ctypes.byref(f),
+        None if c is False else ctypes.byref(c), w.layer_idx, s.q_out.data_ptr(),
+        s.q_out.stride(0), -1, s.err.data_ptr(), stream.cuda_stream)
+
+
+def _check(w, got, want):
+    """The no-alloc result against the workspace call's and against the oracle."""
+    T, Hq, D = w.total_tokens, w.n_q_heads, w.cache.head_dim
+    assert int(got.err.item()) == 0
+    H.assert_close_bf16(H.bits(got.q_out).reshape(T, Hq, D),
+                        H.bits(want.q_out).reshape(T, Hq, D), "q_out vs the workspace call")
+    r = H.oracle_ragged_store(w, w.cache.dtype)
+    assert r.err == 0
+    H.assert_close_bf16(H.bits(got.q_out).reshape(T, Hq, D), r.q_out.reshape(T, Hq, D),
+                        "q_out vs the oracle")
+    rope = H.rope_cols(D, w.rope.rope_dim)
+    H.compare_paged_cache(w.cache, H.bits(got.storage), H.bits(want.storage), r.written,
+                          w.layer_idx, rope, "cache vs the workspace call")
+    H.compare_paged_cache(w.cache, H.bits(got.storage), r.storage, r.written, w.layer_idx, rope,
+                          "cache vs the oracle")
+
+
+def test_noalloc_store_matches_the_store_with_a_workspace_and_the_oracle(G):
+    import rope_paged_kv_b200 as rs
     lib = rs.raw_library()
     stream = torch.cuda.current_stream()
     for seed in (21, 22):  # two calls in a row, on different inputs
@@ -40,19 +76,36 @@ def test_noalloc_store_matches_the_store_with_a_workspace():
         want.sched = rs.sched_workspace(G.DEV)
         G.launch_ragged(w, want)
         got = G.stage_ragged(w)
-        f, c = got.freqs.c(), got.kv.c()
-        st = lib.rope_split_store_paged_ragged_noalloc(
-            got.qkv.data_ptr(), got.qkv.stride(0), -1, w.total_tokens, w.n_q_heads,
-            got.offs.data_ptr(), got.offs.shape[0] - 1, ctypes.byref(f), ctypes.byref(c),
-            w.layer_idx, got.q_out.data_ptr(), got.q_out.stride(0), -1, got.err.data_ptr(),
-            stream.cuda_stream)
-        assert st == rs.OK
+        assert _noalloc(lib, w, got, stream) == rs.OK
         torch.cuda.synchronize()
-        assert int(got.err.item()) == int(want.err.item()) == 0
         assert not want.sched.any().item()
-        T, Hq, D = w.total_tokens, w.n_q_heads, w.cache.head_dim
-        H.assert_close_bf16(H.bits(got.q_out).reshape(T, Hq, D),
-                            H.bits(want.q_out).reshape(T, Hq, D), "q_out")
-        written = H.oracle_ragged_store(w, w.cache.dtype).written
-        H.compare_paged_cache(w.cache, H.bits(got.storage), H.bits(want.storage), written,
-                              w.layer_idx, H.rope_cols(D, w.rope.rope_dim), "cache")
+        _check(w, got, want)
+
+
+def test_noalloc_store_allocates_nothing_and_rejected_calls_queue_nothing(G):
+    import rope_paged_kv_b200 as rs
+    lib = rs.raw_library()
+    stream = torch.cuda.current_stream()
+    w = _workload(23)
+    want = G.stage_ragged(w)
+    want.sched = rs.sched_workspace(G.DEV)
+    G.launch_ragged(w, want)
+    staged = [G.stage_ragged(w) for _ in range(4)]
+    assert _noalloc(lib, w, staged[0], stream) == rs.OK  # the first call does the set-up
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for s in staged[1:]:
+        assert _noalloc(lib, w, s, stream) == rs.OK
+    # no tokens: returns at once; a rejected call (no cache descriptor) returns its status
+    assert _noalloc(lib, w, staged[1], stream, total_tokens=0) == rs.OK
+    assert _noalloc(lib, w, staged[1], stream, kv=False) == rs.ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0, "device memory was allocated"
+    # every call after the rejected one is still right
+    last = G.stage_ragged(w)
+    assert _noalloc(lib, w, last, stream) == rs.OK
+    torch.cuda.synchronize()
+    for s in staged + [last]:
+        assert np.array_equal(H.bits(s.q_out), H.bits(staged[0].q_out))
+        assert np.array_equal(H.bits(s.storage), H.bits(staged[0].storage))
+    _check(w, last, want)
