@@ -4,9 +4,9 @@ Bit-exact: page/slot placement, V copies, columns neither normed nor rotated, ev
 byte the operation must not touch, the radd sums, the device error bits.  Rotated / normed
 values: |gpu - oracle| <= max(1 ulp of the oracle value in the element type, 1e-3).
 Sizes: the five named workloads at full size (with the claimed-tail token schedule the
-benchmark uses, under the default launch-overlap mode; test_gpu_schedule.py shows every mode,
-the benchmark's included, bit-identical) plus small cases that span several tiles and
-ragged tails, and the edge cases.
+benchmark uses, under the default launch-overlap mode and the benchmark's own; the
+test_gpu_schedule.py cases show every mode bit-identical) plus small cases that span several
+tiles and ragged tails, and the edge cases.
 """
 import json
 import os
@@ -42,8 +42,9 @@ def _slot_rows(kv, storage_bits, cache_lengths, lengths, layer_idx):
                      W.token_slots(kv, list(cache_lengths), list(lengths))])
 
 
-def check_ragged(G, w, s, exact_norm_cols=False, multiply_before_cast=True):
-    r = H.oracle_ragged_store(w, w.cache.dtype, multiply_before_cast)
+def check_ragged(G, w, s, exact_norm_cols=False, multiply_before_cast=True, r=None):
+    if r is None:
+        r = H.oracle_ragged_store(w, w.cache.dtype, multiply_before_cast)
     assert int(s.err.item()) == r.err
     D, T, Hq, Hk = w.cache.head_dim, w.total_tokens, w.n_q_heads, w.cache.n_kv_heads
     norm = w.q_gamma is not None
@@ -77,18 +78,39 @@ def test_tiny_ragged(G):
     assert r.err == 0 and int(r.written.sum()) == 8
 
 
+# The full-size cases run under the default launch-overlap mode and under the one the
+# benchmark times (descriptor arrays read before the wait for the preceding kernels), each
+# compared with the oracle.
+FULL_SIZE_MODES = (1, 2)
+
+
+def _under_modes(run):
+    """run() under every mode of FULL_SIZE_MODES, the process-wide mode restored after."""
+    import rope_paged_kv_b200 as rs
+    before = rs.get_launch_overlap()
+    try:
+        for mode in FULL_SIZE_MODES:
+            rs.set_launch_overlap(mode)
+            run()
+    finally:
+        rs.set_launch_overlap(before)
+
+
 def test_llama3_8b_prefill_full_size(G):
     w = W.llama3_8b_prefill()
-    check_ragged(G, w, G.run_ragged(w))
+    r = H.oracle_ragged_store(w, w.cache.dtype)
+    _under_modes(lambda: check_ragged(G, w, G.run_ragged(w), r=r))
 
 
 def test_per_head_norm_full_size(G):
     w = W.per_head_norm()
-    check_ragged(G, w, G.run_ragged(w))
+    r = H.oracle_ragged_store(w, w.cache.dtype)
+    _under_modes(lambda: check_ragged(G, w, G.run_ragged(w), r=r))
 
 
-def _check_dual(G, w, s, multiply_before_cast=True):
-    r = H.oracle_dual(w, multiply_before_cast=multiply_before_cast)
+def _check_dual(G, w, s, multiply_before_cast=True, r=None):
+    if r is None:
+        r = H.oracle_dual(w, multiply_before_cast=multiply_before_cast)
     assert int(s.err.item()) == r.err
     D = w.main_cache.head_dim
     allc = np.ones(D, bool)
@@ -120,11 +142,13 @@ def _check_dual(G, w, s, multiply_before_cast=True):
 
 def test_dual_band_full_size(G):
     w = W.dual_band_minimax()
-    _check_dual(G, w, G.run_dual(w))
+    r = H.oracle_dual(w)
+    _under_modes(lambda: _check_dual(G, w, G.run_dual(w), r=r))
 
 
-def _check_radd(G, w, s):
-    r = H.oracle_radd(w, w.cache.dtype)
+def _check_radd(G, w, s, r=None):
+    if r is None:
+        r = H.oracle_radd(w, w.cache.dtype)
     assert int(s.err.item()) == r.err
     H.assert_bits_equal(H.bits(s.storage), r.storage, "cache after radd")
     return r
@@ -132,11 +156,13 @@ def _check_radd(G, w, s):
 
 def test_radd_full_size(G):
     w = W.radd_minimax()
-    _check_radd(G, w, G.run_radd(w))
+    r = H.oracle_radd(w, w.cache.dtype)
+    _under_modes(lambda: _check_radd(G, w, G.run_radd(w), r=r))
 
 
-def _check_bshd(G, w, s, pristine):
-    r = H.oracle_bshd(w, w.cache.dtype)
+def _check_bshd(G, w, s, pristine, r=None):
+    if r is None:
+        r = H.oracle_bshd(w, w.cache.dtype)
     assert int(s.err.item()) == r.err
     D = w.cache.head_dim
     fpc = H.rope_cols(D, w.rope.rope_dim, w.rope.rope_col_offset)
@@ -154,11 +180,15 @@ def _check_bshd(G, w, s, pristine):
 
 def test_decode_bshd_full_size(G):
     w = W.decode_bshd()
-    s = G.stage_bshd(w)
-    pristine = s.storage.clone()
-    G.launch_bshd(w, s)
-    torch.cuda.synchronize()
-    _check_bshd(G, w, s, pristine)
+    r = H.oracle_bshd(w, w.cache.dtype)
+
+    def run():
+        s = G.stage_bshd(w)
+        pristine = s.storage.clone()
+        G.launch_bshd(w, s)
+        torch.cuda.synchronize()
+        _check_bshd(G, w, s, pristine, r=r)
+    _under_modes(run)
 
 
 # ------------------------------------------------------------------------ edge cases --
