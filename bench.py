@@ -3,24 +3,27 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one rope_split_store_paged_ragged call (RoPE of Q and K, split, paged K/V store)
-over the Llama-3-8B-shaped ragged prefill batch: 32 Q / 8 KV heads, head_dim 128, 8
-sequences with seeded lengths U[256, 2048], page_size 128, half-split RoPE, bf16.  Inputs are
-resident in HBM and larger than L2: the steps rotate over three separate copies of the
-workload (about 0.8 GB), launched back to back, so no step finds its inputs in L2 and every
-step pays for writing back the dirty lines its predecessor left.  `value` = tokens
-processed by all ranks / the max over ranks of the summed per-step device time (CUDA events
-on the launching stream).  Under torchrun every rank runs its own replica
-of the workload (its own seeded batch: weak scaling, no collective on the data path).
+One step = one fused_dual_qk_rmsnorm_rope_paged call (per-head RMSNorm, partial RoPE, the
+split into Q outputs and paged K/V stores, two bands in one launch) over the dual-band batch:
+a main band of 64 Q / 8 KV heads and an index band of 8 Q / 1 K-only head, head_dim 128,
+RoPE over 64 columns, 32768 tokens over 64 sequences, page_size 128 / 64, bf16: the largest
+of the named workloads (1.49 GB of algorithmic traffic a call).  Inputs are resident in HBM
+and larger than L2: the steps rotate over three separate copies of the workload, launched
+back to back, so no step finds its inputs in L2 and every step pays for writing back the
+dirty lines its predecessor left.  `value` = tokens processed by all ranks / the max over
+ranks of the summed per-step device time (CUDA events on the launching stream).  Under
+torchrun every rank runs its own replica of the workload (its own seeded batch: weak
+scaling, no collective on the data path).  --workload NAME times another named workload as
+the main line.
 
 Also printed (same JSON line): `e2e` (the same step through the Python binding with the
-inputs copied from pinned host memory and q_out copied back inside the timed region),
+inputs copied from pinned host memory and the result copied back inside the timed region),
 `roofline` (algorithmic bytes of one launch / mean launch time, against the measured HBM
 copy bandwidth), `cpu_baseline` (the CPU oracle on one host core and on all of them),
-`clocks` (nvidia-smi samples during the timed region), `launch_modes` (the headline under
-every launch-overlap mode and token schedule) and `entry_points` (every other named
-workload through its entry point, at N=1; the latency-bound ones also as launches captured
-in a CUDA graph).
+`clocks` (nvidia-smi and NVML samples during the timed region), `launch_modes` (the main
+workload under every launch-overlap mode and token schedule) and `entry_points` (every other
+named workload through its entry point, at N=1; the latency-bound ones also as launches
+captured in a CUDA graph).
 """
 from __future__ import annotations
 
@@ -39,6 +42,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fused RoPE+KV-store tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+HEADLINE = "dual_band_minimax"  # the largest single-GPU configuration
 UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20   # L2 flush for the decode case's cold-cache figure
 REPLICAS = 3               # rotating copies of a workload: inputs larger than L2
@@ -46,7 +50,6 @@ FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/rope_store.cu", "rope_paged_kv_b200/csrc/banded.cuh",
                   "rope_paged_kv_b200/csrc/common.cuh", "rope_paged_kv_b200/csrc/pipeline.cuh",
                   "rope_paged_kv_b200/csrc/device_utils.cuh"]
-PROFILE = "profiles/rope_split_store_paged_ragged_llama3_8b_prefill.md"
 
 
 def parse_args():
@@ -55,7 +58,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="llama3_8b_prefill",
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=HEADLINE,
                     help="the named workload timed as the main line (default: the headline)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the other entry points and the CPU baseline")
@@ -67,8 +70,9 @@ def parse_args():
                     help="token schedule of the staged kernels: claimed tail (a scheduling "
                          "workspace) or static")
     ap.add_argument("--profile-range", action="store_true",
-                    help="bracket the timed steps with cudaProfilerStart / Stop, so that a "
-                         "range-replay profiler measures them as one back-to-back range")
+                    help="after the timed steps, replay them once more as one CUDA graph "
+                         "between cudaProfilerStart / Stop, so that a range-replay profiler "
+                         "measures them as one back-to-back range")
     return ap.parse_args()
 
 
@@ -92,10 +96,15 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback (earlier measurement on this pool)"
 
 
-def profiled_traffic():
-    """dram bytes per launch from the committed ncu summary, if it was taken on the current
-    kernel sources (else None)."""
-    p = os.path.join(ROOT, PROFILE)
+def profile_summary(workload):
+    """The committed ncu summary of a workload's kernel."""
+    return os.path.join(ROOT, "profiles", f"{WORKLOADS[workload]}_{workload}.md")
+
+
+def profiled_traffic(workload):
+    """dram bytes per launch from the workload's committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = profile_summary(workload)
     if not os.path.exists(p):
         return None
     text = open(p).read()
@@ -146,8 +155,10 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self, t0: float, t1: float):
-        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+    def summary(self, t0: float, t1: float, extra=()):
+        """Clocks over the timed region [t0, t1]: this sampler's samples there plus `extra`
+        (NVML samples taken across the region), else every sample taken."""
+        inside = [s for s in list(self.samples) + list(extra) if t0 <= s[0] <= t1]
         use = inside or self.samples
         if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
@@ -155,6 +166,49 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(s[1] for s in use),
                 "sm_max_mhz": max(s[2] for s in use), "reasons": reasons,
                 "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+class NvmlPoller:
+    """NVML samples of the SM clock and the clock-event reasons, taken as fast as NVML
+    answers (0.5 ms apart) between start() and stop(): a timed region of a few milliseconds
+    still gets samples, which the nvidia-smi sampler's period may miss."""
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
+
+    def __init__(self, uuid):
+        self.samples, self.h, self.nv = [], None, None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        except Exception:
+            self.h = None
+
+    def _loop(self):
+        nv, h = self.nv, self.h
+        while not self.done:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                return
+            self.samples.append((time.time(), float(mhz), float(mx),
+                                 [n for n, b in self.BITS.items() if bits & b]))
+            time.sleep(0.0005)
+
+    def start(self):
+        self.done = False
+        if self.h is not None:
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+
+    def stop(self):
+        self.done = True
+        if self.h is not None:
+            self.thread.join(timeout=5)
+        return self.samples
 
 
 # ------------------------------------------------------------- algorithmic bytes --
@@ -597,14 +651,14 @@ def run_ours(args):
     K = args.steps
     barrier()
     torch.cuda.synchronize()
+    poller = NvmlPoller(f"GPU-{uuid}" if uuid is not None else "")
+    poller.start()
     t0 = time.time()
-    if args.profile_range:
-        torch.cuda.profiler.start()
     dev_ms = time_steps(torch, steps, K, stream)
-    if args.profile_range:
-        torch.cuda.profiler.stop()
     t1 = time.time()
+    nvml_samples = poller.stop()
     barrier()
+    prof = profile_range(torch, args, dev, w, use_sched, n_rep, K) if args.profile_range else None
 
     K_e2e = max(1, min(K, 200))
     time_e2e(torch, cases[:2], 3, stream)
@@ -657,11 +711,10 @@ def run_ours(args):
                         "next step's copy-in)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic() if args.workload == "llama3_8b_prefill"
-                     else None,
+                     "traffic": profiled_traffic(args.workload),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": case.alg_bytes,
                      "kernel": KERNELS[args.workload]},
-        "clocks": sampler.summary(t0, t1),
+        "clocks": sampler.summary(t0, t1, nvml_samples),
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
@@ -669,7 +722,41 @@ def run_ours(args):
         line["launch_modes"] = modes
     if extras:
         line["entry_points"] = extras
+    if prof is not None:
+        line["profile_range"] = prof
     print(json.dumps(line), flush=True)
+
+
+def profile_range(torch, args, dev, w, use_sched, n_rep, K):
+    """The K timed steps again, captured in one CUDA graph (on a stream of their own, over
+    fresh copies of the workload) and replayed once between cudaProfilerStart / Stop, so
+    that a range-replay profiler sees them back to back, free of host launch gaps.  Returns
+    the replay's device time, measured outside any profiler pass that adds overhead."""
+    gs = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(gs):
+        cases = [make_case(args.workload, 0, dev, w, use_sched) for _ in range(n_rep)]
+        for i in range(max(3, n_rep)):
+            cases[i % n_rep].step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=gs):
+        for i in range(K):
+            cases[i % n_rep].step()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(gs):
+        g.replay()  # warm-up replay
+        torch.cuda.synchronize()
+        torch.cuda.profiler.start()
+        e0.record(gs)
+        g.replay()
+        e1.record(gs)
+        torch.cuda.synchronize()
+        torch.cuda.profiler.stop()
+    ms = e0.elapsed_time(e1)
+    del g, cases
+    torch.cuda.empty_cache()
+    return {"launches": K, "graph_replay_us": round(ms * 1e3, 2),
+            "us_per_launch": round(ms * 1e3 / K, 2)}
 
 
 KERNELS = {"llama3_8b_prefill": "banded_store_kernel<bf16, head_dim 128, no norm>",
@@ -800,15 +887,35 @@ def run_entry_points(torch, dev, stream, headline, peak, use_sched, reps=30):
     return out
 
 
-def oracle_token_shares(w, n):
-    """The oracle's calls for a ragged store batch split into n contiguous token ranges.
+def _token_ranges(offs, cls_list, T, n):
+    """For n contiguous token ranges of a ragged batch: (r0, r1, sequences touched, row
+    offsets of the range's pieces, each piece's starting position per cache-length list)."""
+    out = []
+    for i in range(n):
+        r0, r1 = T * i // n, T * (i + 1) // n
+        rows, o, c = [], [0], [[] for _ in cls_list]
+        for b in range(len(offs) - 1):
+            a, e = max(offs[b], r0), min(offs[b + 1], r1)
+            if a < e:
+                rows.append(b)
+                o.append(o[-1] + e - a)
+                for k, cls in enumerate(cls_list):
+                    c[k].append(cls[b] + a - offs[b])
+        out.append((r0, r1, rows, o, c))
+    return out
 
-    Each range is a ragged batch of its own: a sequence's piece keeps its page-table row and
+
+def oracle_token_shares(w, n):
+    """The oracle's calls for a ragged batch (a ragged store or the dual-band launch) split
+    into n contiguous token ranges.
+
+    Each range is a ragged batch of its own: a sequence's piece keeps its page-table rows and
     starts at the position of its first token (the sequence's cache length plus the piece's
     offset in it), so the pieces write exactly the slots and Q rows the whole batch writes.
-    The calls share one host copy of the cache (their slots are disjoint) and views of the
-    input and Q output; each returns the oracle's error bits.  Running them one after another
-    or at once gives the same bytes as one call on the whole batch."""
+    The calls share one host copy of each cache (their slots are disjoint) and views of the
+    input and Q outputs; each returns the oracle's error bits.  Running them one after
+    another or at once gives the same bytes as one call on the whole batch.  Returns the
+    calls, the cache storage(s) and the Q output(s)."""
     import dataclasses
     import functools
 
@@ -816,53 +923,101 @@ def oracle_token_shares(w, n):
     import torch
 
     import oracle
+    import workloads as W
     from oracle import runners as R
     T = w.total_tokens
-    store, qkv, q_out = R.bits(w.cache.storage), R.bits(w.qkv), R.bits(w.q_out)
     rope = R.oracle_rope(w.rope)
     offs = [int(x) for x in w.offsets.tolist()]
-    cls = [int(x) for x in w.cache.cache_lengths.tolist()]
+
+    def sub(kv, rows, c):
+        return dataclasses.replace(kv, page_table=kv.page_table[rows].contiguous(),
+                                   cache_lengths=torch.tensor(c, dtype=torch.int32))
     calls = []
-    for i in range(n):
-        r0, r1 = T * i // n, T * (i + 1) // n
-        rows, o, c = [], [0], []
-        for b in range(len(offs) - 1):
-            a, e = max(offs[b], r0), min(offs[b + 1], r1)
-            if a < e:
-                rows.append(b)
-                o.append(o[-1] + e - a)
-                c.append(cls[b] + a - offs[b])
-        kv = dataclasses.replace(w.cache, page_table=w.cache.page_table[rows].contiguous(),
-                                 cache_lengths=torch.tensor(c, dtype=torch.int32))
+    if isinstance(w, W.DualBand):
+        inp, qm, qi = R.bits(w.input), R.bits(w.q_main_out), R.bits(w.q_index_out)
+        ms, ist = R.bits(w.main_cache.storage), R.bits(w.index_cache.storage)
+        g = [R.bits(x) for x in w.gammas]
+        cls = [w.cache_lengths_of(w.main_cache), w.cache_lengths_of(w.index_cache)]
+        for r0, r1, rows, o, c in _token_ranges(offs, cls, T, n):
+            main = oracle.Band(inp[r0:r1], *w.main_cols, w.main_q_heads,
+                               R.oracle_paged(sub(w.main_cache, rows, c[0]), ms), g[0], g[1],
+                               w.main_eps, qm[r0:r1])
+            index = oracle.Band(inp[r0:r1], *w.index_cols, w.index_q_heads,
+                                R.oracle_paged(sub(w.index_cache, rows, c[1]), ist), g[2],
+                                g[3], w.index_eps, qi[r0:r1])
+            calls.append(functools.partial(oracle.fused_dual_qk_rmsnorm_rope_paged, main,
+                                           index, np.array(o, dtype=np.uint32), rope,
+                                           w.weight_offset, True, w.layer_idx))
+        return calls, (ms, ist), (qm, qi)
+    store, qkv, q_out = R.bits(w.cache.storage), R.bits(w.qkv), R.bits(w.q_out)
+    cls = [[int(x) for x in w.cache.cache_lengths.tolist()]]
+    for r0, r1, rows, o, c in _token_ranges(offs, cls, T, n):
         calls.append(functools.partial(oracle.rope_split_store_paged_ragged, qkv[r0:r1],
                                        w.n_q_heads, np.array(o, dtype=np.uint32), rope,
-                                       R.oracle_paged(kv, store), w.layer_idx, q_out[r0:r1]))
+                                       R.oracle_paged(sub(w.cache, rows, c[0]), store),
+                                       w.layer_idx, q_out[r0:r1]))
     return calls, store, q_out
 
 
-def cpu_baseline(workload, min_seconds=10.0, max_reps=20):
-    """The oracle as it stands (single-threaded C, double precision) on the headline
-    workload's batch (the same seeded batch rank 0 measured), and the same oracle run on
-    every core this process may use: one thread per core over contiguous token ranges (the
-    C calls release the interpreter lock)."""
-    from concurrent.futures import ThreadPoolExecutor
-
+def oracle_call(w):
+    """One oracle call on a whole ragged batch (a ragged store or the dual-band launch)."""
     import workloads as W
     from oracle import runners as R
-    if workload != "llama3_8b_prefill":
+    return R.oracle_dual(w) if isinstance(w, W.DualBand) else R.oracle_ragged_store(w)
+
+
+def batch_prefix(workload, n_tokens, seed=1):
+    """A batch shaped like the named ragged workload over the first sequences of its batch
+    (the last one cut short) holding about n_tokens tokens: the bounded sample the CPU
+    baselines time.  Returns (batch, sequences used)."""
+    import workloads as W
+    full = make_workload(workload, 0)
+    lengths, left = [], n_tokens
+    for n in full.lengths:
+        if left <= 0:
+            break
+        lengths.append(min(n, left))
+        left -= lengths[-1]
+    k = len(lengths)
+    if workload == "dual_band_minimax":
+        cls = full.cache_lengths_of(full.main_cache)[:k]
+        return W.dual_band(seed, lengths=lengths, cache_lengths=cls, main_q_heads=64,
+                           main_kv_heads=8, index_q_heads=8, index_kv_heads=1, head_dim=128,
+                           main_page_size=128, index_page_size=64, rope_dim=64, theta=1e4,
+                           interleaved=True, max_seq_len=8192, name=full.name), k
+    return W.ragged_store(seed, lengths=lengths, cache_lengths=[0] * k, n_q_heads=32,
+                          n_kv_heads=8, head_dim=128, page_size=128, rope_dim=128, theta=5e5,
+                          interleaved=False, max_seq_len=8192, width=64, name=full.name), k
+
+
+CPU_BASELINE_WORKLOADS = ("llama3_8b_prefill", "dual_band_minimax")
+
+
+def cpu_baseline(workload, min_seconds=10.0, max_reps=20, max_tokens=12288):
+    """The oracle as it stands (single-threaded C, double precision) on the workload's batch
+    (the same seeded batch rank 0 measured, its first max_tokens tokens when larger), and the
+    same oracle run on every core this process may use: one thread per core over contiguous
+    token ranges (the C calls release the interpreter lock)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    if workload not in CPU_BASELINE_WORKLOADS:
         return None
-    w = W.llama3_8b_prefill(seed=0)
+    w = make_workload(workload, 0)
+    what = f"the full benchmark batch ({w.total_tokens} tokens)"
+    if w.total_tokens > max_tokens:
+        w, k = batch_prefix(workload, max_tokens, seed=0)
+        what = (f"the benchmark batch's first {w.total_tokens} tokens (from {k} of its "
+                f"sequences)")
     reps, t_total = 0, 0.0
     while t_total < min_seconds and reps < max_reps:
         t = time.perf_counter()
-        R.oracle_ragged_store(w)
+        oracle_call(w)
         t_total += time.perf_counter() - t
         reps += 1
     out = {"value": round(w.total_tokens * reps / t_total, 1), "unit": UNIT, "cores": 1,
            "kind": "oracle",
-           "sample": f"the full benchmark batch ({w.total_tokens} tokens), {reps} passes, "
-                     f"{t_total:.1f} s; single-threaded C, double precision (host copy-in "
-                     f"of the arrays included)"}
+           "sample": f"{what}, {reps} passes, {t_total:.1f} s; single-threaded C, double "
+                     f"precision (host copy-in of the arrays included)"}
     cores = len(os.sched_getaffinity(0))
     if cores > 1:
         n = min(cores, w.total_tokens)
@@ -877,7 +1032,7 @@ def cpu_baseline(workload, min_seconds=10.0, max_reps=20):
         assert not any(errs)
         out["all_cores"] = {
             "value": round(w.total_tokens * reps_p / t_par, 1), "unit": UNIT, "cores": n,
-            "sample": f"the same batch in {n} contiguous token ranges, one thread per core "
+            "sample": f"the same tokens in {n} contiguous token ranges, one thread per core "
                       f"(sched_getaffinity), {reps_p} passes, {t_par:.1f} s"}
     return out
 
@@ -892,34 +1047,20 @@ def run_reference(args):
         return
     from concurrent.futures import ThreadPoolExecutor
 
-    import workloads as W
-    from oracle import runners as R
-    full = W.llama3_8b_prefill(seed=0)
+    workload = args.workload if args.workload in CPU_BASELINE_WORKLOADS else HEADLINE
+    full = make_workload(workload, 0)
     steps, warm = args.steps, max(3, args.warmup)
     cores = len(os.sched_getaffinity(0))
 
-    def sample_of(lengths):
-        return W.ragged_store(1, lengths=lengths, cache_lengths=[0] * len(lengths),
-                              n_q_heads=32, n_kv_heads=8, head_dim=128, page_size=128,
-                              rope_dim=128, theta=5e5, interleaved=False, max_seq_len=8192,
-                              width=64)
-
     # size each step's sample (the batch's first tokens, sequence by sequence, the last one
     # cut short) so that the whole run stays within ~2 minutes whatever the step count
-    one = sample_of(full.lengths[:1])
+    one, _ = batch_prefix(workload, 256)
     t = time.perf_counter()
-    R.oracle_ragged_store(one)
+    oracle_call(one)
     per_token = (time.perf_counter() - t) / one.total_tokens / max(1.0, 0.5 * cores)
     budget = 120.0 / (steps + warm)
-    left = int(min(full.total_tokens, max(64, budget / per_token)))
-    lengths = []
-    for n in full.lengths:
-        if left <= 0:
-            break
-        lengths.append(min(n, left))
-        left -= lengths[-1]
-    n_seq = len(lengths)
-    w = sample_of(lengths)
+    w, n_seq = batch_prefix(workload, int(min(full.total_tokens,
+                                              max(64, budget / per_token))))
     n = min(cores, w.total_tokens)
     calls, _, _ = oracle_token_shares(w, n)
     with ThreadPoolExecutor(n) as ex:
@@ -934,15 +1075,15 @@ def run_reference(args):
             step()
             total += time.perf_counter() - t
     value = w.total_tokens * steps / total
-    sample = (f"the batch's first {w.total_tokens} tokens (from {n_seq} of its 8 sequences) "
-              f"per step, split into {n} contiguous token ranges on {n} threads (one per "
-              f"core); C oracle, double precision")
+    sample = (f"the batch's first {w.total_tokens} tokens (from {n_seq} of its "
+              f"{len(full.lengths)} sequences) per step, split into {n} contiguous token "
+              f"ranges on {n} threads (one per core); C oracle, double precision")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
         "n_gpus": args.gpus, "steps": steps, "warmup": warm,
         "ms_per_step": round(total / steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": full.name, "entry_point": "rope_split_store_paged_ragged",
+        "config": {"workload": full.name, "entry_point": WORKLOADS[workload],
                    "sample": sample},
         "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": n, "kind": "oracle",
                          "sample": sample},

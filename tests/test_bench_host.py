@@ -131,3 +131,36 @@ def test_algorithmic_bytes_of_the_named_workloads():
     assert bench.bytes_bshd(b) == 256 * (20736 - 256) + frb
     g = W.mla_kv_a_proj()
     assert bench.bytes_gemv(g) == (576 * 7168 + 7168 + 512 + 576) * 2
+
+
+@pytest.mark.parametrize("n", [1, 4])
+def test_oracle_token_shares_of_the_dual_band_write_what_the_whole_batch_writes(n):
+    # the same for the two-band launch, whose bands keep caches and page sizes of their own
+    from concurrent.futures import ThreadPoolExecutor
+
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    from oracle import runners as R
+    w = W.dual_band(33, lengths=[30, 1, 45], cache_lengths=[3, 70, 0], main_q_heads=4,
+                    main_kv_heads=2, index_q_heads=2, index_kv_heads=1, head_dim=64,
+                    main_page_size=16, index_page_size=8, rope_dim=32, theta=1e4,
+                    interleaved=True, max_seq_len=256)
+    want = R.oracle_dual(w)
+    assert want.err == 0
+    calls, (ms, ist), (qm, qi) = bench.oracle_token_shares(w, n)
+    with ThreadPoolExecutor(n) as ex:
+        assert list(ex.map(lambda f: f(), calls)) == [0] * n
+    assert np.array_equal(ms, want.main_storage) and np.array_equal(ist, want.index_storage)
+    assert np.array_equal(qm, want.q_main_out) and np.array_equal(qi, want.q_index_out)
+
+
+def test_batch_prefix_takes_the_first_sequences_of_the_batch():
+    sys.path.insert(0, ROOT)
+    import bench
+    full = bench.make_workload("dual_band_minimax", 0)
+    w, k = bench.batch_prefix("dual_band_minimax", 5000)
+    assert w.total_tokens == 5000 and w.lengths[:-1] == full.lengths[:k - 1]
+    assert w.lengths[-1] <= full.lengths[k - 1]
+    assert w.cache_lengths_of(w.main_cache) == full.cache_lengths_of(full.main_cache)[:k]
