@@ -351,16 +351,16 @@ const char *rope_status_string(rope_status_t status);
 rope_status_t rope_set_launch_overlap(int32_t mode);
 int32_t rope_get_launch_overlap(void);
 
-/* A diagnostic of the failure path, not an operation of the pages: the most polls a
- * pipeline wait inside the staged kernels (the three paged stores, kv_cache_radd,
- * matmul_fused_partial_rmsnorm) makes before it gives up, for launches that follow,
- * process-wide.  A wait that gives up sets ROPE_DEVERR_TIMEOUT, the CTA leaves its loops and
- * the call returns incomplete.  0 (the default) means about 2^30 polls or 2 s, whichever
- * ends first; the waits that let a CTA's in-flight copies land before it exits keep that
- * default whatever is set here.  A small limit (1) makes waits run out in normal operation:
- * a test of the timeout path. */
-rope_status_t rope_set_wait_limit(uint32_t polls);
-uint32_t rope_get_wait_limit(void);
+/* A diagnostic of the failure path, not an operation of the pages.  With timeout_us > 0,
+ * every launch that follows of the staged kernels (the three paged stores, kv_cache_radd,
+ * matmul_fused_partial_rmsnorm) starts with one wait that nothing ever completes (an
+ * mbarrier no thread arrives at), bounded by timeout_us instead of the usual 2 s.  When it
+ * runs out the kernel does what it does when any of its waits runs out: it sets
+ * ROPE_DEVERR_TIMEOUT, every CTA leaves its loops after letting its in-flight copies land
+ * (those waits keep the full limit), and the call returns incomplete.  0 (the default) turns
+ * it off.  Process-wide; timeout_us above 1000000 is ROPE_ERR_INVALID_ARG. */
+rope_status_t rope_set_stall_test(uint32_t timeout_us);
+uint32_t rope_get_stall_test(void);
 
 #ifdef __cplusplus
 }

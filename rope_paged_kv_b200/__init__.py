@@ -111,13 +111,13 @@ _lib.matmul_fused_partial_rmsnorm.argtypes = [
 _lib.rope_set_launch_overlap.argtypes = [_i32]
 _lib.rope_get_launch_overlap.argtypes = []
 _lib.rope_get_launch_overlap.restype = _i32
-_lib.rope_set_wait_limit.argtypes = [_u32]
-_lib.rope_get_wait_limit.argtypes = []
-_lib.rope_get_wait_limit.restype = _u32
+_lib.rope_set_stall_test.argtypes = [_u32]
+_lib.rope_get_stall_test.argtypes = []
+_lib.rope_get_stall_test.restype = _u32
 for _f in ("rope_split_store_paged_ragged", "fused_qk_rmsnorm_rope_paged",
            "fused_dual_qk_rmsnorm_rope_paged", "qk_rope_bshd_continuous", "kv_cache_radd",
            "rope_set_launch_overlap", "rope_split_store_paged_ragged_noalloc",
-           "rope_set_wait_limit",
+           "rope_set_stall_test",
            "matmul_fused_partial_rmsnorm"):
     getattr(_lib, _f).restype = ctypes.c_int
 _lib.rope_status_string.argtypes = [ctypes.c_int]
@@ -178,14 +178,15 @@ def get_launch_overlap() -> int:
     return int(_lib.rope_get_launch_overlap())
 
 
-def set_wait_limit(polls: int) -> None:
-    """The most polls a pipeline wait makes before it gives up (0: the default), for the
-    launches that follow (process-wide): a diagnostic of the timeout path."""
-    _check(_lib.rope_set_wait_limit(int(polls)), "rope_set_wait_limit")
+def set_stall_test(timeout_us: int) -> None:
+    """A diagnostic of the timeout path (process-wide): with timeout_us > 0 the staged
+    kernels of the launches that follow start with a wait that nothing completes, bounded by
+    timeout_us; when it runs out they take the path of a wait that runs out.  0: off."""
+    _check(_lib.rope_set_stall_test(int(timeout_us)), "rope_set_stall_test")
 
 
-def get_wait_limit() -> int:
-    return int(_lib.rope_get_wait_limit())
+def get_stall_test() -> int:
+    return int(_lib.rope_get_stall_test())
 
 
 def _row_stride(t: torch.Tensor) -> int:

@@ -149,38 +149,47 @@ __device__ __forceinline__ uint32_t e4m3_exact(float v, float inv, float s) {
   return above == (sgn == 0u) ? ch : cl;
 }
 
+// E4M3 codes of v0..v3 * inv as one word (code i in byte i), each converted once (nearest,
+// ties to even, saturating)
+__device__ __forceinline__ uint32_t e4m3_scaled4(float v0, float v1, float v2, float v3,
+                                                 float inv) {
+  return __nv_cvt_float2_to_fp8x2(make_float2(v0 * inv, v1 * inv), __NV_SATFINITE, __NV_E4M3) |
+         (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(v2 * inv, v3 * inv), __NV_SATFINITE,
+                                            __NV_E4M3)
+             << 16;
+}
+
+// Whether s is 2^k with both s and 1/s normal floats: then v * (1/s) is v / s exactly, up to
+// an overflow or underflow that E4M3 saturates or rounds to zero either way.
+__device__ __forceinline__ int pow2_scale(float s) {
+  const uint32_t b = __float_as_uint(s), e = (b >> 23) & 0xffu;
+  return (b & 0x807fffffu) == 0u && e >= 1u && e <= 253u;
+}
+
 // E4M3 codes of v0..v3 / s as one word (code i in byte i), each rounded exactly once as
-// e4m3_exact does: the codes of the four quotients moved two ulps down and up in magnitude
-// come from two packed conversions each, and agree as words unless a rounding boundary lies
-// between them for some value (or a value is not finite or saturates), which sends that
-// word through e4m3_exact value by value.
+// e4m3_exact does.  The conversion of q = v * inv is the answer unless q is not the exact
+// quotient (v - q * s, exact in one fused multiply-add, is not zero) and lies within two
+// ulps of a rounding boundary of the normal E4M3 grid (bit 19 of the mantissa set, bits
+// 18..0 clear: a midpoint between codes), or below it (|q| < 2^-6, the subnormal codes);
+// such a value, which is rare, goes through e4m3_exact.  With a power-of-two scale q is
+// always exact.
 __device__ __forceinline__ uint32_t e4m3_exact4(float v0, float v1, float v2, float v3,
-                                                 float inv, float s) {
+                                                float inv, float s) {
   const float v[4] = {v0, v1, v2, v3};
-  uint32_t lo[4], hi[4];
-  bool edge = false;
+  float q[4];
+  bool slow = false;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t b = __float_as_uint(v[i] * inv), mag = b & 0x7fffffffu;
-    lo[i] = mag < 2u ? b : b - 2u;  // sign and magnitude: two ulps toward zero
-    hi[i] = b + 2u;                 // and away from it
-    edge |= mag >= 0x7f7ffffeu;
+    q[i] = v[i] * inv;
+    const uint32_t b = __float_as_uint(q[i]), e = (b >> 23) & 0xffu;
+    const bool near = ((b & 0xfffffu) - 0x7fffeu) <= 4u;
+    slow |= (near || e < 121u) && fmaf(-q[i], s, v[i]) != 0.f;
   }
-  const uint32_t cl = __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(lo[0]),
-                                                           __uint_as_float(lo[1])),
-                                               __NV_SATFINITE, __NV_E4M3) |
-                      (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(lo[2]),
-                                                                     __uint_as_float(lo[3])),
-                                                         __NV_SATFINITE, __NV_E4M3)
-                          << 16;
-  const uint32_t ch = __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(hi[0]),
-                                                           __uint_as_float(hi[1])),
-                                               __NV_SATFINITE, __NV_E4M3) |
-                      (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(hi[2]),
-                                                                     __uint_as_float(hi[3])),
-                                                         __NV_SATFINITE, __NV_E4M3)
-                          << 16;
-  if (cl == ch && !edge) return cl;
+  if (!slow)
+    return __nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3) |
+           (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE,
+                                              __NV_E4M3)
+               << 16;
   return e4m3_exact(v[0], inv, s) | e4m3_exact(v[1], inv, s) << 8 |
          e4m3_exact(v[2], inv, s) << 16 | e4m3_exact(v[3], inv, s) << 24;
 }
@@ -198,7 +207,7 @@ struct BandedParams {
   uint32_t *err;
   float weight_offset;
   int32_t mbc;  // multiply_before_cast: 0 rounds the normalised value before the gamma multiply
-  uint32_t wait_polls;  // the most polls of a pipeline wait (drains keep kSpinLimit)
+  uint32_t stall_test_ns;  // > 0: the launch starts with a wait nothing completes (a test)
   // dynamic shared memory layout
   int32_t S, stage_bytes, f_row_bytes, staged, elem_bytes;
   int32_t bar_off, meta_off, gamma_off, offs_off, items_off;
@@ -462,20 +471,13 @@ __device__ __forceinline__ void rotate_lane(const LaneFreqs<2 * H2, INTER> &fr,
 }
 
 // Where a band's rows go in the extended-output instantiation: Q rows rounded into q_dtype
-// at shared address qo (when q_conv), K rows as E4M3 codes of value * kinv at k8 (when kv8),
-// others back in place; row r of the band's block sits at blk + r * D * element size.
+// at shared address qo (when q_conv), K rows as E4M3 codes of value * kinv at k8 and V rows
+// as the exactly rounded codes of value / vs at v8 (when kv8), others back in place; row r
+// of the band's block sits at blk + r * D * element size.
 struct BandOut {
-  uint32_t blk, qo, k8;
-  int q_conv, q_dtype, q_eb, kv8, n_q;
-  float kinv;
-};
-
-// gamma + weight_offset of a lane's columns for one row kind (the shared address of its
-// gamma row), kept in registers across rows while the kind does not change
-template <int N>
-struct LaneGamma {
-  uint32_t addr;
-  float a[N], b[N];
+  uint32_t blk, qo, k8, v8;
+  int q_conv, q_dtype, q_eb, kv8, n_q, n_kv, v_pow2;
+  float kinv, vinv, vs;
 };
 
 // J head rows of a staged token, listed at it[0], it[stride], ...: optionally normalised
@@ -483,14 +485,12 @@ struct LaneGamma {
 // rotated with the token's table row F (INTER: the interleaved layout), written back in
 // place.  The J rows' dependency chains are interleaved.  EF: `fr` holds the table row
 // already; else it is read here, after the norm (so that it and the gammas are never live
-// together).  KG: `lg` keeps the gamma last read across calls; else gammas are read per
-// chunk.  EXT: outputs as `bo` says.
-template <int J, typename T, int D, bool NORM, int L, bool INTER, bool EXT, bool EF, bool KG>
+// together).  EXT: outputs as `bo` says.
+template <int J, typename T, int D, bool NORM, int L, bool INTER, bool EXT, bool EF>
 __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t *it, int stride,
                                           uint32_t st, uint32_t gq, uint32_t gk, float eps,
                                           int mbc, const unsigned char *F,
-                                          LaneFreqs<Vec<T>::N, INTER> &fr,
-                                          LaneGamma<Vec<T>::N> &lg, const BandOut &bo) {
+                                          LaneFreqs<Vec<T>::N, INTER> &fr, const BandOut &bo) {
   using VT = Vec<T>;
   constexpr int N = VT::N, H2 = N / 2, EB = (int)sizeof(T);
   uint32_t row[J], g[J];
@@ -530,16 +530,13 @@ __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t
     for (int msk = L / 2; msk > 0; msk >>= 1)
 #pragma unroll
       for (int j = 0; j < J; ++j) r[j] += __shfl_xor_sync(cl.gmask, r[j], msk);
-    float ga_[N], gb_[N];  // gamma + weight_offset of the lane's columns, read once per kind
-    float(&ga)[N] = KG ? lg.a : ga_;
-    float(&gb)[N] = KG ? lg.b : gb_;
+    float ga[N], gb[N];  // gamma + weight_offset of the lane's columns, read once per kind
 #pragma unroll
     for (int j = 0; j < J; ++j) {
       r[j] = rsqrtf(r[j] * (1.0f / D) + eps);
-      if (KG ? g[j] != lg.addr : (j == 0 || g[j] != g[j - 1])) {
+      if (j == 0 || g[j] != g[j - 1]) {
         lds_f32<N>(g[j] + cl.ca * 4, cl.li, ga);
         lds_f32<N>(g[j] + cl.cb * 4, cl.li, gb);
-        if (KG) lg.addr = g[j];
       }
       if (mbc) {  // x * gamma now; the scalar r after the rotation
 #pragma unroll
@@ -605,38 +602,65 @@ __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t
   }
 }
 
-// A band's slots [lo, hi) of a consumer thread's head rows, JM at a time.  Without the norm
-// (and, if so built, one row at a time) the table row is read once here, for every chunk.
-#ifndef ROPE_ONE_ROW_EARLY_FREQS
-#define ROPE_ONE_ROW_EARLY_FREQS 1
-#endif
-#ifndef ROPE_ONE_ROW_KEEP_GAMMA
-#define ROPE_ONE_ROW_KEEP_GAMMA 0
-#endif
+// The V rows of an FP8 band among a consumer thread's slots [lo, hi): the lane's two
+// vectors of each row encoded as E4M3 codes of value / scale, each rounded once (with a
+// power-of-two scale the product with its reciprocal is the exact quotient, and one
+// conversion rounds it).
+template <typename T, int D>
+__device__ __forceinline__ void v_rows(const ConsumerLane &cl, const uint32_t *item, int stride,
+                                       int lo, int hi, uint32_t st, const BandOut &bo) {
+  using VT = Vec<T>;
+  constexpr int N = VT::N, EB = (int)sizeof(T);
+#pragma unroll 1
+  for (int u = lo; u < hi; ++u) {
+    const uint32_t row = st + (item[u * stride] & kItemOffMask);
+    const int rb = (int)(row - bo.blk) / (D * EB);
+    const uint32_t vrow = bo.v8 + (uint32_t)((rb - bo.n_q - bo.n_kv) * D);
+    float x[2][N];
+    VT::widen(lds_v4(row + cl.ca * EB), x[0]);
+    VT::widen(lds_v4(row + cl.cb * EB), x[1]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t a = vrow + (h ? cl.cb : cl.ca);
+      const uint32_t w0 = bo.v_pow2 ? e4m3_scaled4(x[h][0], x[h][1], x[h][2], x[h][3], bo.vinv)
+                                    : e4m3_exact4(x[h][0], x[h][1], x[h][2], x[h][3], bo.vinv,
+                                                  bo.vs);
+      if constexpr (N == 8) {
+        const uint32_t w1 =
+            bo.v_pow2 ? e4m3_scaled4(x[h][4], x[h][5], x[h][6], x[h][7], bo.vinv)
+                      : e4m3_exact4(x[h][4], x[h][5], x[h][6], x[h][7], bo.vinv, bo.vs);
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(w0), "r"(w1) : "memory");
+      } else {
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(a), "r"(w0) : "memory");
+      }
+    }
+  }
+}
+
+// A band's slots [lo, hi) of a consumer thread's head rows, JM at a time.  Without the norm,
+// or one row at a time, the table row is read once here, for every chunk.
 template <int JM, typename T, int D, bool NORM, int L, bool INTER, bool EXT>
 __device__ __forceinline__ void rows_band(const ConsumerLane &cl, const uint32_t *item, int stride,
                                           int lo, int hi, uint32_t st, uint32_t gq, uint32_t gk,
                                           float eps, int mbc, const unsigned char *F,
-                                          LaneGamma<Vec<T>::N> &lg, const BandOut &bo) {
-  // one row at a time: the table row once per band and token, gamma kept across rows
-  constexpr bool EF = !NORM || (JM == 1 && ROPE_ONE_ROW_EARLY_FREQS);
-  constexpr bool KG = NORM && JM == 1 && ROPE_ONE_ROW_KEEP_GAMMA;
+                                          const BandOut &bo) {
+  constexpr bool EF = !NORM || JM == 1;
   LaneFreqs<Vec<T>::N, INTER> fr;
   if constexpr (EF) load_lane_freqs<Vec<T>::N, INTER>(fr, cl, F);
   int u = lo;
 #pragma unroll 1
   for (; u + JM <= hi; u += JM)
-    rows_step<JM, T, D, NORM, L, INTER, EXT, EF, KG>(cl, item + u * stride, stride, st, gq, gk,
-                                                    eps, mbc, F, fr, lg, bo);
+    rows_step<JM, T, D, NORM, L, INTER, EXT, EF>(cl, item + u * stride, stride, st, gq, gk, eps,
+                                                 mbc, F, fr, bo);
   if constexpr (JM >= 3) {
     if (hi - u == 2)
-      rows_step<2, T, D, NORM, L, INTER, EXT, EF, KG>(cl, item + u * stride, stride, st, gq, gk,
-                                                     eps, mbc, F, fr, lg, bo);
+      rows_step<2, T, D, NORM, L, INTER, EXT, EF>(cl, item + u * stride, stride, st, gq, gk, eps,
+                                                  mbc, F, fr, bo);
   }
   if constexpr (JM >= 2) {
     if (hi - u == 1)
-      rows_step<1, T, D, NORM, L, INTER, EXT, EF, KG>(cl, item + u * stride, stride, st, gq, gk,
-                                                     eps, mbc, F, fr, lg, bo);
+      rows_step<1, T, D, NORM, L, INTER, EXT, EF>(cl, item + u * stride, stride, st, gq, gk, eps,
+                                                  mbc, F, fr, bo);
   }
 }
 
@@ -675,6 +699,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
   uint32_t *s_cl = s_offs + (p.batch + 1);
   uint32_t *s_items = reinterpret_cast<uint32_t *>(smem + p.items_off);
   __shared__ int s_abort;
+  __shared__ __align__(8) uint64_t s_never;  // no thread ever arrives here
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) grid_dep_launch_dependents();
@@ -684,6 +709,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
       mbar_init(&done[s], kConsumerWarps);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(&s_never, 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -713,7 +739,15 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
   const int n_local = (p.T - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
   unsigned char *stages = smem;
 
-  if (warp == 0) {
+  if (p.stall_test_ns != 0 && warp >= 2) {
+    // A test of the timeout path (stall_test_ns > 0): the consumers wait on a barrier that
+    // no thread ever arrives at, for at most stall_test_ns; when the wait runs out they do
+    // what a pipeline wait that runs out makes them do.
+    if (!mbar_wait(&s_never, 0, &s_abort, p.stall_test_ns) && lane == 0) {
+      s_abort = 1;
+      raise(p.err, ROPE_DEVERR_TIMEOUT);
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------------ producer --
     const bool dyn = p.sched != nullptr;
     const int n_static = static_tokens(p.T, n_local, dyn);
@@ -767,7 +801,7 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
         mj.stop = 0;
         const int s = issued % p.S;
         if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
+          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
             aborted = true;
           } else {
             meta[s] = mj;
@@ -837,102 +871,46 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
       }
     }
     // stop marker: the next stage carries no token
+    bool marked = false;  // the stop marker went into stage issued % S
     if (!aborted && lane == 0) {
       const int s = issued % p.S;
-      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
+      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
         aborted = true;
       } else {
         meta[s].stop = 1;
         mbar_arrive(&full[s]);
+        marked = true;
       }
     }
     aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
-    if (aborted && lane == 0) {
-      s_abort = 1;
-      raise(p.err, ROPE_DEVERR_TIMEOUT);
-      // let the loads already issued land before the CTA's shared memory goes away
-      for (int ii = max(0, issued - p.S); ii < issued; ++ii) {
+    if (lane == 0) {
+      if (aborted) {
+        s_abort = 1;
+        raise(p.err, ROPE_DEVERR_TIMEOUT);
+      }
+      // let the loads issued land before the CTA's shared memory goes away: only the last S
+      // can be in flight (a stage is reloaded only once the storer released it); in a run
+      // that did not give up the consumers have waited for them already.  The stop marker
+      // took the stage of token issued - S one phase further, and that token was stored
+      // before the stage was handed back: its phase is not waited for (its parity now names
+      // the marker's next, unfinished phase).
+      for (int ii = max(0, issued - p.S + (marked ? 1 : 0)); ii < issued; ++ii) {
         int never = 0;
         mbar_wait(&full[ii % p.S], (ii / p.S) & 1, &never);
       }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------------- storer --
-    // With an FP8 cache that takes V, every lane of the warp first encodes the staged V rows
-    // (nothing else reads them): E4M3 codes of value / scale, each rounded exactly once.
-    const bool venc = EXT && ((p.band[0].kv8 && p.band[0].n_v) ||
-                              (p.n_bands > 1 && p.band[1].kv8 && p.band[1].n_v));
-    if (lane == 0 || venc) {
+    if (lane == 0) {
       int n_done = 0;  // tokens stored
-      float vs[2] = {1.f, 1.f}, vinv[2] = {1.f, 1.f};
       for (int i = 0;; ++i) {
         const int s = i % p.S;
-        if constexpr (EXT) {
-          if (venc) {
-            const bool got =
-                __all_sync(0xffffffffu, mbar_wait(&full[s], (i / p.S) & 1, &s_abort, p.wait_polls));
-            if (!got) {
-              if (lane == 0) {
-                s_abort = 1;
-                raise(p.err, ROPE_DEVERR_TIMEOUT);
-              }
-              break;
-            }
-            if (i == 0) {  // after the producer's wait for the preceding kernels
-#pragma unroll
-              for (int k = 0; k < 2; ++k)
-                if (k < p.n_bands && (k ? p.band[1] : p.band[0]).kv8 &&
-                    (k ? p.band[1] : p.band[0]).n_v) {
-                  vs[k] = __ldg((k ? p.band[1] : p.band[0]).v_scale);
-                  vinv[k] = 1.f / vs[k];
-                }
-            }
-            if (!meta[s].stop) {
-              const uint32_t st = smem_addr(stages) + (uint32_t)(s * p.stage_bytes);
-#pragma unroll
-              for (int k = 0; k < 2; ++k) {
-                if (k >= p.n_bands || !meta[s].ok[k]) continue;
-                const BandDev &bd = k ? p.band[1] : p.band[0];
-                if (!bd.kv8 || !bd.n_v) continue;
-                const uint32_t vblk = st + (uint32_t)(bd.smem_off + (bd.n_q + bd.n_kv) * D * EB);
-                const uint32_t v8 = st + (uint32_t)bd.v8_off;
-                const int nvec = bd.n_v * D / N;
-                for (int vv = lane; vv < nvec; vv += 32) {
-                  float x[N];
-                  VT::widen(lds_v4(vblk + vv * 16), x);
-                  uint32_t w[N / 4];
-#pragma unroll
-                  for (int q = 0; q < N / 4; ++q)
-                    w[q] = e4m3_exact4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3],
-                                       vinv[k], vs[k]);
-                  if constexpr (N == 8) {
-                    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(v8 + vv * N),
-                                 "r"(w[0]), "r"(w[N / 4 - 1])
-                                 : "memory");
-                  } else {
-                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(v8 + vv * N), "r"(w[0])
-                                 : "memory");
-                  }
-                }
-              }
-              fence_proxy_async_smem();  // the bulk copies below read these codes
-            }
-            __syncwarp();
-          }
+        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort)) {
+          s_abort = 1;
+          raise(p.err, ROPE_DEVERR_TIMEOUT);
+          break;
         }
-        int stop = 0;
-        if (lane == 0) {
-          if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
-            s_abort = 1;
-            raise(p.err, ROPE_DEVERR_TIMEOUT);
-            stop = 2;
-          } else if (meta[s].stop) {
-            stop = 1;
-          }
-        }
-        if (venc) stop = __shfl_sync(0xffffffffu, stop, 0);
-        if (stop) break;
-        if (lane != 0) continue;
+        if (meta[s].stop) break;
         n_done = i + 1;
         const uint32_t tok = (uint32_t)meta[s].tok;
         const unsigned char *st = stages + (size_t)s * p.stage_bytes;
@@ -977,11 +955,9 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
           mbar_arrive(&empty[(i - kStoreLag) % p.S]);
         }
       }
-      if (lane == 0) {
-        bulk_wait_read<0>();
-        for (int i = max(0, n_done - kStoreLag); i < n_done; ++i) mbar_arrive(&empty[i % p.S]);
-        bulk_wait<0>();
-      }
+      bulk_wait_read<0>();
+      for (int i = max(0, n_done - kStoreLag); i < n_done; ++i) mbar_arrive(&empty[i % p.S]);
+      bulk_wait<0>();
     }
   } else {
     // ------------------------------------------------------------------ consumers --
@@ -1022,34 +998,41 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
     const int fa = inter ? ca - rp.off : 2 * (ca - rp.off);
     const int fb = cb - rp.off;
     const ConsumerLane cl{li, ca, cb, fa, fb, rp.dtype, inter, rot_a, rot_b, gmask};
-    // this thread's head rows of a token, decoded once into shared memory: rows of band 0
-    // in slots [0, u_end0), of band 1 in [u_end0, u_end1)
+    // this thread's head rows of a token, decoded once into shared memory: band 0's Q and K
+    // rows in slots [0, qk0), its V rows (FP8 caches only) in [qk0, end0); band 1's in
+    // [beg1, qk1) and [qk1, end1)
     const int n_items = (p.work_total + G - 1) / G;
     uint32_t *item = s_items + ctid;  // slot u at item[u * kConsumers]
-    int u_end0 = 0, u_end1 = 0;
+    int qk0 = 0, end0 = 0, beg1 = -1, qk1 = 0, end1 = 0;
     for (int u = 0; u < n_items; ++u) {
       const int j = grp + u * G;
       uint32_t w = 0;
       if (j < p.work_total) {
         const int band = j >= p.work0 ? 1 : 0;
         const BandDev &bd = band ? p.band[1] : p.band[0];
-        const int r = j - (band ? p.work0 : 0);  // Q heads then K heads: stage rows 0..
-        const int kind = r < bd.n_q ? 0 : 1;
+        const int r = j - (band ? p.work0 : 0);  // Q heads, K heads, V heads: stage rows 0..
+        const int kind = r < bd.n_q ? 0 : r < bd.n_q + bd.n_kv ? 1 : 2;
         const uint32_t soff = (uint32_t)(bd.smem_off + r * D * EB);
         w = kItemAct | (uint32_t)band << kItemBandShift | (uint32_t)kind << kItemKindShift | soff;
-        if (band == 0) u_end0 = u + 1;
-        u_end1 = u + 1;
+        if (band == 0) {
+          if (kind < 2) qk0 = u + 1;
+          end0 = u + 1;
+        } else {
+          if (beg1 < 0) beg1 = qk1 = u;
+          if (kind < 2) qk1 = u + 1;
+          end1 = u + 1;
+        }
       }
       item[u * kConsumers] = w;
     }
+    if (beg1 < 0) beg1 = qk1 = end1 = end0;
     const uint32_t stages_a = smem_addr(stages);
     const uint32_t gamma_a = smem_addr(s_gamma);
-    float kinv[2] = {1.f, 1.f};  // 1 / scale of FP8 K planes
-    LaneGamma<N> lg;             // one-row chunks: the gamma last read, kept across rows
-    lg.addr = ~0u;
+    // FP8 planes: 1 / scale of K, scale and 1 / scale of V
+    float kinv[2] = {1.f, 1.f}, vsc[2] = {1.f, 1.f}, vinv[2] = {1.f, 1.f};
     for (int i = 0;; ++i) {
       const int s = i % p.S;
-      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
+      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
         if (lane == 0) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);
@@ -1062,33 +1045,46 @@ __global__ void __launch_bounds__(pipe_threads<CW>(), pipe_min_ctas<CW, NORM>())
         break;
       }
       if (EXT && i == 0) {  // after the producer's wait for the preceding kernels
-        if (p.band[0].kv8) kinv[0] = 1.f / __ldg(p.band[0].k_scale);
-        if (p.n_bands > 1 && p.band[1].kv8) kinv[1] = 1.f / __ldg(p.band[1].k_scale);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const BandDev &bd = k ? p.band[1] : p.band[0];
+          if (k < p.n_bands && bd.kv8) {
+            kinv[k] = 1.f / __ldg(bd.k_scale);
+            if (bd.n_v) {
+              vsc[k] = __ldg(bd.v_scale);
+              vinv[k] = 1.f / vsc[k];
+            }
+          }
+        }
       }
       const uint32_t st = stages_a + (uint32_t)(s * p.stage_bytes);
       const int ok0 = meta[s].ok[0], ok1 = meta[s].ok[1];
 #pragma unroll 1
       for (int band = 0; band < p.n_bands; ++band) {
-        const int lo = band ? u_end0 : 0, hi = band ? u_end1 : u_end0;
+        const int lo = band ? beg1 : 0, qk = band ? qk1 : qk0, hi = band ? end1 : end0;
         if (lo >= hi || !(band ? ok1 : ok0)) continue;
         const BandDev &bd = band ? p.band[1] : p.band[0];
-        // lanes with nothing to do leave their bytes in place, unless they go elsewhere
-        if (!busy && !(EXT && (bd.q_conv || bd.kv8))) continue;
-        const unsigned char *F = stages + (size_t)s * p.stage_bytes + bd.f_off;
-        const float eps = bd.eps;
-        const uint32_t gq = gamma_a + (uint32_t)(band * 2 * D * 4), gk = gq + D * 4;
         BandOut bo{};
         if constexpr (EXT) {
           bo = BandOut{st + (uint32_t)bd.smem_off, st + (uint32_t)bd.qo_off,
-                       st + (uint32_t)bd.k8_off, bd.q_conv, bd.q_dtype, bd.q_eb, bd.kv8, bd.n_q,
-                       kinv[band]};
+                       st + (uint32_t)bd.k8_off,   st + (uint32_t)bd.v8_off,
+                       bd.q_conv, bd.q_dtype, bd.q_eb, bd.kv8, bd.n_q, bd.n_kv,
+                       pow2_scale(band ? vsc[1] : vsc[0]), band ? kinv[1] : kinv[0],
+                       band ? vinv[1] : vinv[0],
+                       band ? vsc[1] : vsc[0]};
+          if (qk < hi) v_rows<T, D>(cl, item, kConsumers, qk, hi, st, bo);
         }
+        // lanes with nothing to do leave their bytes in place, unless they go elsewhere
+        if (lo >= qk || (!busy && !(EXT && (bd.q_conv || bd.kv8)))) continue;
+        const unsigned char *F = stages + (size_t)s * p.stage_bytes + bd.f_off;
+        const float eps = bd.eps;
+        const uint32_t gq = gamma_a + (uint32_t)(band * 2 * D * 4), gk = gq + D * 4;
         if (inter)
-          rows_band<JM, T, D, NORM, L, true, EXT>(cl, item, kConsumers, lo, hi, st, gq, gk, eps,
-                                                 p.mbc, F, lg, bo);
+          rows_band<JM, T, D, NORM, L, true, EXT>(cl, item, kConsumers, lo, qk, st, gq, gk, eps,
+                                                 p.mbc, F, bo);
         else
-          rows_band<JM, T, D, NORM, L, false, EXT>(cl, item, kConsumers, lo, hi, st, gq, gk,
-                                                  eps, p.mbc, F, lg, bo);
+          rows_band<JM, T, D, NORM, L, false, EXT>(cl, item, kConsumers, lo, qk, st, gq, gk,
+                                                  eps, p.mbc, F, bo);
       }
       fence_proxy_async_smem();  // the storer's bulk copies read what was written here
       __syncwarp();

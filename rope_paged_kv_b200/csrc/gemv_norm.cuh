@@ -32,7 +32,7 @@ struct GemvParams {
   uint32_t *err;
   int32_t overlap;
   int32_t row_bytes;  // k * element size, padded to 16: a row's place in shared memory
-  uint32_t wait_polls;  // the most polls of the load wait (the drain keeps kSpinLimit)
+  uint32_t stall_test_ns;  // > 0: the launch starts with a wait nothing completes (a test)
 };
 
 template <typename T>
@@ -71,10 +71,12 @@ __global__ void __launch_bounds__(kGemvThreads)
   __shared__ int s_last;
   __shared__ __align__(8) uint64_t bar;
   __shared__ int s_abort;
+  __shared__ __align__(8) uint64_t s_never;  // no thread ever arrives here
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) grid_dep_launch_dependents();
   if (STAGED && tid == 0) {
     mbar_init(&bar, 1);
+    mbar_init(&s_never, 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -91,6 +93,13 @@ __global__ void __launch_bounds__(kGemvThreads)
   if constexpr (STAGED) {
     __syncthreads();  // the barrier is initialised
     const uint32_t kb = (uint32_t)p.k * sizeof(T);
+    // A test of the timeout path (stall_test_ns > 0): the loading thread first waits on a
+    // barrier that no thread ever arrives at, for at most stall_test_ns; when that runs out
+    // the CTA takes the path of a load wait that runs out.
+    if (tid == 0 && p.stall_test_ns != 0 && !mbar_wait(&s_never, 0, &s_abort, p.stall_test_ns)) {
+      s_abort = 1;
+      raise(p.err, ROPE_DEVERR_TIMEOUT);
+    }
     if (tid == 0 && kb > 0) {
       mbar_arrive_expect_tx(&bar, kb * (uint32_t)(rows + 1));
       bulk_g2s(smem, x, kb, &bar);
@@ -99,7 +108,7 @@ __global__ void __launch_bounds__(kGemvThreads)
                  kb, &bar);
     }
     bool ok = true;
-    if (kb > 0 && !mbar_wait(&bar, 0, &s_abort, p.wait_polls)) {
+    if (kb > 0 && !mbar_wait(&bar, 0, &s_abort)) {
       ok = false;
       if (lane == 0) raise(p.err, ROPE_DEVERR_TIMEOUT);
     }

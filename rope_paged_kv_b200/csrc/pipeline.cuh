@@ -62,31 +62,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return done != 0;
 }
 
-// The same test without the hardware's suspend: returns at once.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // Wait until the phase of `bar` with parity `parity` has completed.  Gives up (returns
-// false) after kWaitLimitNs of wall time or max_polls polls (kSpinLimit unless a caller
-// asks for fewer), or early once *abort is set by another thread of the CTA.  A caller's
-// smaller poll limit polls without the hardware's suspend (mbarrier.try_wait may sleep a
-// while before it fails), so that such a wait runs out after max_polls quick tests.
+// false) after limit_ns of wall time (kWaitLimitNs unless a caller asks for less) or
+// kSpinLimit polls, or early once *abort is set by another thread of the CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
                                           const volatile int *abort,
-                                          uint32_t max_polls = kSpinLimit) {
+                                          uint64_t limit_ns = kWaitLimitNs) {
   uint64_t t0 = 0;
-  const bool quick = max_polls < kSpinLimit;
-  for (uint32_t it = 0; it < max_polls; ++it) {
-    if (quick ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  for (uint32_t it = 0; it < kSpinLimit; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
 #if ROPE_WAIT_BACKOFF_NS > 0
     if (it >= 2) __nanosleep(ROPE_WAIT_BACKOFF_NS);  // leave the issue slots to busy warps
 #endif
@@ -95,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
       const uint64_t now = global_ns();
       if (t0 == 0)
         t0 = now;
-      else if (now - t0 > kWaitLimitNs)
+      else if (now - t0 > limit_ns)
         return false;
     }
   }

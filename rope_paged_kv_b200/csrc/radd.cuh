@@ -25,7 +25,7 @@ struct RaddParams {
   int32_t S, stage_bytes, staged, kv_contig;  // kv_contig: a token's heads are adjacent
   int32_t bar_off, meta_off, offs_off;
   int32_t overlap;  // launch-overlap mode (kOverlap*)
-  uint32_t wait_polls;  // the most polls of a pipeline wait (drains keep kSpinLimit)
+  uint32_t stall_test_ns;  // > 0: the launch starts with a wait nothing completes (a test)
   uint32_t *sched;  // claim counter + finished CTAs, or nullptr for a static schedule
 };
 
@@ -51,6 +51,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
   uint32_t *s_offs = reinterpret_cast<uint32_t *>(smem + p.offs_off);
   uint32_t *s_cl = s_offs + (p.batch + 1);
   __shared__ int s_abort;
+  __shared__ __align__(8) uint64_t s_never;  // no thread ever arrives here
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) grid_dep_launch_dependents();
@@ -60,6 +61,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
       mbar_init(&done[s], CW);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(&s_never, 1);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -83,7 +85,15 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
   const int64_t hidden = (int64_t)p.n_kv * D;
   const uint32_t row_bytes = (uint32_t)(hidden * EB);  // one plane's heads of one token
 
-  if (warp == 0) {
+  if (p.stall_test_ns != 0 && warp >= 2) {
+    // A test of the timeout path (stall_test_ns > 0): the consumers wait on a barrier that
+    // no thread ever arrives at, for at most stall_test_ns; when the wait runs out they do
+    // what a pipeline wait that runs out makes them do.
+    if (!mbar_wait(&s_never, 0, &s_abort, p.stall_test_ns) && lane == 0) {
+      s_abort = 1;
+      raise(p.err, ROPE_DEVERR_TIMEOUT);
+    }
+  } else if (warp == 0) {
     const bool dyn = p.sched != nullptr;
     const int n_static = static_tokens(p.T, n_local, dyn);
     const int dyn0 = n_static * (int)gridDim.x;  // first claimed token
@@ -121,7 +131,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
         mj.tok = __shfl_sync(0xffffffffu, m.tok, j);
         const int s = issued % p.S;
         if (lane == 0) {
-          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
+          if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
             aborted = true;
           } else {
             meta[s] = mj;
@@ -175,20 +185,26 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
         issue(m, cnt);
       }
     }
+    bool marked = false;  // the stop marker went into stage issued % S
     if (!aborted && lane == 0) {  // stop marker
       const int s = issued % p.S;
-      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort, p.wait_polls)) {
+      if (!mbar_wait(&empty[s], ((issued / p.S) & 1) ^ 1, &s_abort)) {
         aborted = true;
       } else {
         meta[s].stop = 1;
         mbar_arrive(&full[s]);
+        marked = true;
       }
     }
     aborted = __shfl_sync(0xffffffffu, aborted ? 1 : 0, 0) != 0;
-    if (aborted && lane == 0) {
-      s_abort = 1;
-      raise(p.err, ROPE_DEVERR_TIMEOUT);
-      for (int ii = max(0, issued - p.S); ii < issued; ++ii) {
+    if (lane == 0) {
+      if (aborted) {
+        s_abort = 1;
+        raise(p.err, ROPE_DEVERR_TIMEOUT);
+      }
+      // let the loads issued land before the CTA's shared memory goes away (the last S;
+      // after the stop marker, not token issued - S, stored before its stage was reused)
+      for (int ii = max(0, issued - p.S + (marked ? 1 : 0)); ii < issued; ++ii) {
         int never = 0;
         mbar_wait(&full[ii % p.S], (ii / p.S) & 1, &never);
       }
@@ -199,7 +215,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
       int n_done = 0;
       for (int i = 0;; ++i) {
         const int s = i % p.S;
-        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
+        if (!mbar_wait(&done[s], (i / p.S) & 1, &s_abort)) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);
           break;
@@ -238,7 +254,7 @@ __global__ void __launch_bounds__(radd_threads<CW>(), 1) radd_kernel(const __gri
     const int rows = 2 * p.n_kv;
     for (int i = 0;; ++i) {
       const int s = i % p.S;
-      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort, p.wait_polls)) {
+      if (!mbar_wait(&full[s], (i / p.S) & 1, &s_abort)) {
         if (lane == 0) {
           s_abort = 1;
           raise(p.err, ROPE_DEVERR_TIMEOUT);

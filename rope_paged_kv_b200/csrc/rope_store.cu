@@ -64,8 +64,11 @@ static int passes(const BandedParams &p, int D, int cw) {
 }
 
 static ShapeId pick_shape(const BandedParams &p, int D, bool norm) {
-  // few head rows without norm, or Q converted to another type: the light shape (the V rows
-  // of an FP8 cache are encoded by the storer warp, not by the consumers)
+  // few head rows without norm (Q, K and, for an FP8 cache, V), or Q converted to another
+  // type: the light shape
+#ifdef ROPE_FP8_MID
+  if (!norm && p.band[0].kv8) return kMid;
+#endif
   if (!norm && (p.work_total <= 64 || p.band[0].q_conv)) return kLight;
 #ifdef ROPE_NORM_ALWAYS_MID
   if (norm) return kMid;
@@ -81,13 +84,9 @@ static const BandedShape &shape_of(ShapeId id) {
 
 // launch-overlap mode of every launch that follows (rope_set_launch_overlap)
 static std::atomic<int> g_overlap{kOverlapPdl};
-// the most polls of a pipeline wait in the launches that follow (rope_set_wait_limit; 0: the
-// default)
-static std::atomic<uint32_t> g_wait_polls{0};
-static uint32_t wait_polls() {
-  const uint32_t w = g_wait_polls.load(std::memory_order_relaxed);
-  return w ? w : kSpinLimit;
-}
+// the stall test of the launches that follow (rope_set_stall_test): 0 off, else the limit of
+// the wait nothing completes, in nanoseconds
+static std::atomic<uint32_t> g_stall_test_ns{0};
 
 // Launch `kern` with one parameter block; modes 1 and 2 launch it as a programmatic
 // dependent of the previous kernel in the stream.
@@ -552,7 +551,8 @@ static rope_status_t prepare_ragged_store(const void *qkv, int64_t qkv_row_strid
                 q_out_dtype);
   if (s != ROPE_OK) return s;
   p.n_bands = 1;
-  p.work0 = p.work_total = (int32_t)(Hq + Hk);  // the head rows the consumers take: Q and K
+  // the head rows the consumers take: Q and K, and V when it is encoded for an FP8 cache
+  p.work0 = p.work_total = (int32_t)(Hq + Hk + (p.band[0].kv8 ? Hk : 0));
   p.offs = input_row_offsets;
   p.batch = batch;
   p.T = total_tokens;
@@ -560,7 +560,7 @@ static rope_status_t prepare_ragged_store(const void *qkv, int64_t qkv_row_strid
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
-  p.wait_polls = wait_polls();
+  p.stall_test_ns = g_stall_test_ns.load(std::memory_order_relaxed);
   work = p.work_total + Hk > 0;  // V alone (no Q or K heads) is still copied
   return ROPE_OK;
 }
@@ -688,7 +688,8 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
                 q_gamma, k_gamma, epsilon, q_out, q_out_row_stride, dtype, layer_idx, true);
   if (s != ROPE_OK) return s;
   p.n_bands = 1;
-  p.work0 = p.work_total = (int32_t)(Hq + Hk);  // the head rows the consumers take: Q and K
+  // the head rows the consumers take: Q and K, and V when it is encoded for an FP8 cache
+  p.work0 = p.work_total = (int32_t)(Hq + Hk + (p.band[0].kv8 ? Hk : 0));
   p.offs = input_row_offsets;
   p.batch = batch;
   p.T = total_tokens;
@@ -696,7 +697,7 @@ rope_status_t fused_qk_rmsnorm_rope_paged(const void *qkv, int64_t qkv_row_strid
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
-  p.wait_polls = wait_polls();
+  p.stall_test_ns = g_stall_test_ns.load(std::memory_order_relaxed);
   p.weight_offset = round_to_elem(weight_offset, dtype);
   if (p.work_total + Hk == 0) return ROPE_OK;
   return launch_banded(dtype, D, true, p, (cudaStream_t)stream);
@@ -740,7 +741,8 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
                   b->n_q_heads, b->cache, b->q_gamma, b->k_gamma, b->epsilon, b->q_out,
                   b->q_out_row_stride, dtype, layer_idx, true);
     if (s != ROPE_OK) return s;
-    rows[k] = p.band[k].n_q + p.band[k].n_kv;  // the head rows the consumers take
+    // the head rows the consumers take: Q and K, and V when it is encoded for an FP8 cache
+    rows[k] = p.band[k].n_q + p.band[k].n_kv + (p.band[k].kv8 ? p.band[k].n_v : 0);
   }
   p.n_bands = n_bands;
   p.work0 = rows[0];
@@ -752,7 +754,7 @@ rope_status_t fused_dual_qk_rmsnorm_rope_paged(const rope_norm_band_t *main_band
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
-  p.wait_polls = wait_polls();
+  p.stall_test_ns = g_stall_test_ns.load(std::memory_order_relaxed);
   p.weight_offset = round_to_elem(weight_offset, dtype);
   if (p.work_total == 0) return ROPE_OK;
   return launch_banded(dtype, D, true, p, (cudaStream_t)stream);
@@ -835,7 +837,7 @@ rope_status_t kv_cache_radd(const void *a, int64_t a_row_stride, int32_t total_t
   p.err = err_word;
   p.sched = sched;
   p.overlap = g_overlap.load(std::memory_order_relaxed);
-  p.wait_polls = wait_polls();
+  p.stall_test_ns = g_stall_test_ns.load(std::memory_order_relaxed);
   p.kv_contig = kv->head_stride == D ? 1 : 0;
   const size_t smem = layout_radd(p, D, eb);
   if (smem > 227 * 1024) return ROPE_ERR_UNSUPPORTED;
@@ -911,7 +913,7 @@ rope_status_t matmul_fused_partial_rmsnorm(const void *input, const void *weight
   p.err = err_word;
   p.row_bytes = (int32_t)round_up((int64_t)k * eb, 16);
   p.overlap = g_overlap.load(std::memory_order_relaxed);
-  p.wait_polls = wait_polls();
+  p.stall_test_ns = g_stall_test_ns.load(std::memory_order_relaxed);
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == ROPE_DTYPE_BF16) return launch_gemv_t<__nv_bfloat16>(p, st);
   if (dtype == ROPE_DTYPE_F16) return launch_gemv_t<__half>(p, st);
@@ -927,11 +929,14 @@ rope_status_t rope_set_launch_overlap(int32_t mode) {
 
 int32_t rope_get_launch_overlap(void) { return g_overlap.load(std::memory_order_relaxed); }
 
-rope_status_t rope_set_wait_limit(uint32_t polls) {
-  g_wait_polls.store(polls, std::memory_order_relaxed);
+rope_status_t rope_set_stall_test(uint32_t timeout_us) {
+  if (timeout_us > 1000000u) return ROPE_ERR_INVALID_ARG;
+  g_stall_test_ns.store(timeout_us * 1000u, std::memory_order_relaxed);
   return ROPE_OK;
 }
 
-uint32_t rope_get_wait_limit(void) { return g_wait_polls.load(std::memory_order_relaxed); }
+uint32_t rope_get_stall_test(void) {
+  return g_stall_test_ns.load(std::memory_order_relaxed) / 1000u;
+}
 
 }  // extern "C"

@@ -1,13 +1,13 @@
-"""The bounded waits: a pipeline wait that runs out ends the call with ROPE_DEVERR_TIMEOUT
-set instead of hanging, and the context stays usable.
+"""The bounded waits: a wait that runs out ends the call with ROPE_DEVERR_TIMEOUT set
+instead of hanging, and the context stays usable.
 
-rope_set_wait_limit(1) caps every pipeline wait of the staged kernels at one poll, so waits
-run out in normal operation: a consumer's first wait for a stage comes before the producer
-has even resolved its tokens and issued the loads.  The waits that let a CTA's in-flight
-copies land before it exits keep their full limit, so every CTA leaves with its copies
-done.  Each case checks the timeout bit, that the scheduling workspace (or the GEMV's count)
-is back at zero, and then runs the same call with the default limit and compares it with
-the oracle.  No kernel traps or is stopped from outside: the failure is a wait that gives up.
+rope_set_stall_test(100) makes every staged kernel start with a wait on a barrier that no
+thread ever arrives at (a flag that nothing sets), bounded by 100 us: it runs out, and the
+kernel takes the path any wait that runs out takes.  The waits that let a CTA's in-flight
+copies land before it exits keep their full limit, so every CTA leaves with its copies done.
+Each case checks the timeout bit, that the scheduling workspace (or the GEMV's count) is
+back at zero, and then runs the same call with the test off and compares it with the oracle.
+No kernel traps or is stopped from outside: the failure is a wait that gives up.
 """
 import pytest
 import torch
@@ -35,15 +35,16 @@ def _ragged(norm, fp8=False):
 
 
 def _short_waits(run):
-    """run() with every pipeline wait capped at one poll; returns what run() returns."""
+    """run() with the stall test on (a 100 us wait nothing completes); returns what run()
+    returns."""
     import rope_paged_kv_b200 as rs
-    assert rs.get_wait_limit() == 0
-    rs.set_wait_limit(1)
+    assert rs.get_stall_test() == 0
+    rs.set_stall_test(100)
     try:
         out = run()
         torch.cuda.synchronize()  # the call returns: nothing hangs
     finally:
-        rs.set_wait_limit(0)
+        rs.set_stall_test(0)
     return out
 
 
