@@ -47,9 +47,9 @@ UNIT = "tokens/s"
 FLUSH_BYTES = 256 << 20   # L2 flush for the decode case's cold-cache figure
 REPLICAS = 3               # rotating copies of a workload: inputs larger than L2
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/rope_store.cu", "rope_paged_kv_b200/csrc/banded.cuh",
-                  "rope_paged_kv_b200/csrc/common.cuh", "rope_paged_kv_b200/csrc/pipeline.cuh",
-                  "rope_paged_kv_b200/csrc/device_utils.cuh"]
+KERNEL_SOURCES = ["rope_paged_kv_b200/csrc/" + f for f in (
+    "rope_store.cu", "banded.cuh", "radd.cuh", "bshd.cuh", "gemv_norm.cuh", "common.cuh",
+    "pipeline.cuh", "device_utils.cuh")]
 
 
 def parse_args():

@@ -13,16 +13,18 @@
 //                      gives a workspace, chunks claimed from a counter after that (see
 //                      static_tokens); a stop marker in the next stage ends the CTA;
 //   warps 2.., consumers: per token, the Q and K head rows are spread over lane groups of
-//                      L = head_dim / vector lanes; each lane normalises (shuffle reduction
-//                      over its group) and rotates its 16 bytes (a half-split partner's 16
-//                      bytes are read from the stage) and writes them back in place;
+//                      L = head_dim / (2 * vector) lanes; each lane owns two 16-byte vectors
+//                      of a row (for half-split RoPE the two halves of its rotation pairs),
+//                      normalises them (shuffle reduction over its group), rotates them and
+//                      writes them back in place, taking up to three of its rows at once so
+//                      that their dependency chains overlap (rows_step);
 //   warp 1, storer:    once the consumers are done with a token, bulk-copies the stage's Q
 //                      block to q_out and its K and V blocks to the cache page, waits until
 //                      the copies have read the stage, and hands the stage back.
-// V rows never enter registers, except for an FP8 cache.  The extended-output instantiation
-// (EXT) writes some results to stage regions of their own instead of in place: Q rounded
-// into another element type, and the E4M3 codes of K and V for an FP8 cache; the storer
-// copies those regions out.  The row range of a token is the band concatenation
+// V rows never enter registers, except for an FP8 cache, where they are consumer rows too
+// (encoded exactly: e4m3_exact4).  The extended-output instantiation (EXT) writes some
+// results to stage regions of their own instead of in place: Q rounded into another element
+// type, and the E4M3 codes of K and V for an FP8 cache; the storer copies those regions out.  The row range of a token is the band concatenation
 // [Q main | K main | V main | Q index | K index | (V index)].
 #pragma once
 
@@ -316,25 +318,16 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
 }
 
 // Head rows a consumer thread takes at once (overlapping their dependency chains), within
-// the register budget of the shape: light CTAs run three to an SM, the others two (a
-// four-warp norm CTA then has about 168 registers a thread).
+// the register budget of the shape: light CTAs run three to an SM, the others two.  Three
+// for the six-warp norm shape (the per-head norm ran 133, 128 and 117-119 us with one, two
+// and three), one elsewhere (the eight-warp shape has 96 registers, and a store without the
+// norm has short chains).
 #ifndef ROPE_CHUNK_ROWS_NORM
 #define ROPE_CHUNK_ROWS_NORM 3
 #endif
-#ifndef ROPE_CHUNK_ROWS_NORM4
-#define ROPE_CHUNK_ROWS_NORM4 4
-#endif
-#ifndef ROPE_CHUNK_ROWS_ROPE
-#define ROPE_CHUNK_ROWS_ROPE 1
-#endif
-#ifndef ROPE_CHUNK_ROWS_8W
-#define ROPE_CHUNK_ROWS_8W 1
-#endif
 template <int CW, bool NORM>
 __host__ __device__ constexpr int chunk_rows() {
-  return CW >= 8 ? ROPE_CHUNK_ROWS_8W
-                 : !NORM ? ROPE_CHUNK_ROWS_ROPE
-                         : CW <= 4 ? ROPE_CHUNK_ROWS_NORM4 : ROPE_CHUNK_ROWS_NORM;
+  return NORM && CW > 4 && CW < 8 ? ROPE_CHUNK_ROWS_NORM : 1;
 }
 
 // M consecutive float32 values from shared address a (16-byte aligned), read bank-conflict

@@ -188,19 +188,42 @@ __global__ void __launch_bounds__(kGemvThreads)
   __syncthreads();
   if (!s_last) return;
 
-  // the last CTA: every entry to be normalised is in the workspace
+  // the last CTA: every entry to be normalised is in the workspace.  A thread keeps the
+  // entries it reads (and their gammas, read at the same time) for the output, so the
+  // normalisation takes one round trip to the workspace; longer rows loop.
   __threadfence();
-  float ss = 0.f;
-  for (int i = tid; i < p.n_normed; i += kGemvThreads) {
-    const float v = __ldcg(p.ws + i);
-    ss = fmaf(v, v, ss);
-  }
-  ss = block_sum(ss, red1);
-  const float r = rsqrtf(ss / (float)p.n_normed + p.eps);
+  constexpr int kKeep = 4;  // entries a thread keeps: n_normed <= 1024 in one pass
   const T *g = reinterpret_cast<const T *>(p.gamma);
   T *out = reinterpret_cast<T *>(p.normed);
-  for (int i = tid; i < p.n_normed; i += kGemvThreads)
-    out[i] = to_elem<T>(__ldcg(p.ws + i) * r * static_cast<float>(g[i]));
+  if (p.n_normed <= kKeep * kGemvThreads) {
+    float v[kKeep], gv[kKeep];
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k) {
+      const int i = tid + k * kGemvThreads;
+      v[k] = i < p.n_normed ? __ldcg(p.ws + i) : 0.f;
+      gv[k] = i < p.n_normed ? static_cast<float>(g[i]) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k) ss = fmaf(v[k], v[k], ss);
+    ss = block_sum(ss, red1);
+    const float r = rsqrtf(ss / (float)p.n_normed + p.eps);
+#pragma unroll
+    for (int k = 0; k < kKeep; ++k) {
+      const int i = tid + k * kGemvThreads;
+      if (i < p.n_normed) out[i] = to_elem<T>(v[k] * r * gv[k]);
+    }
+  } else {
+    float ss = 0.f;
+    for (int i = tid; i < p.n_normed; i += kGemvThreads) {
+      const float v = __ldcg(p.ws + i);
+      ss = fmaf(v, v, ss);
+    }
+    ss = block_sum(ss, red1);
+    const float r = rsqrtf(ss / (float)p.n_normed + p.eps);
+    for (int i = tid; i < p.n_normed; i += kGemvThreads)
+      out[i] = to_elem<T>(__ldcg(p.ws + i) * r * static_cast<float>(g[i]));
+  }
   if (tid == 0) atomicExch(p.count, 0u);
 }
 

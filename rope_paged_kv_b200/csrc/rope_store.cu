@@ -3,12 +3,13 @@
 // Kernels (see the headers):
 //   banded.cuh  ragged paged store, optional per-head RMSNorm, one or two bands: persistent
 //               CTAs, a producer warp bulk-copying token rows into a shared-memory ring,
-//               four, six or eight consumer warps rotating / normalising in place, a
-//               storer warp bulk-copying the results out;
+//               four, six or eight consumer warps rotating / normalising in place (an FP8
+//               cache's codes to stage regions of their own), a storer warp bulk-copying
+//               the results out;
 //   radd.cuh    in-place cache add on the same staging scheme;
 //   bshd.cuh    decode-shaped BSHD RoPE with in-place K, one CTA per token;
-//   gemv_norm.cuh  one-row GEMV + partial RMSNorm, a few rows of W per CTA, the last CTA
-//               normalising.
+//   gemv_norm.cuh  one-row GEMV + partial RMSNorm, one or a few rows of W per CTA, the last
+//               CTA normalising.
 #include "../../include/rope_store.h"
 #include "banded.cuh"
 #include "bshd.cuh"
@@ -40,9 +41,11 @@ struct BandedShape {
 // <= 64 Q+K head rows a token, no norm
 constexpr BandedShape kLightShape = {ROPE_LIGHT_CW, ROPE_LIGHT_LAG, ROPE_LIGHT_RING};
 // RMSNorm or many heads: six or eight consumer warps, whichever takes fewer passes over a
-// token's head rows (six on a tie: 116.6 vs 119.9 us on the per-head-norm workload, whose
-// 72 rows take three passes either way; eight on the dual-band one, 81 rows in three
-// passes instead of four: 248.4 vs 264.8 us)
+// token's head rows (six on a tie: the per-head-norm workload's 72 rows take three passes
+// either way; eight on the dual-band one, 81 rows in three passes instead of four).  One
+// CTA an SM with ten or twelve consumer warps and an eight-stage ring ran 140-150 us on the
+// per-head norm and 372-389 us on the dual band, against 119 and 248 us: two producers and
+// two storers an SM keep more copies in flight.
 #ifndef ROPE_MID_CW
 #define ROPE_MID_CW 6
 #define ROPE_MID_LAG 0
@@ -66,13 +69,7 @@ static int passes(const BandedParams &p, int D, int cw) {
 static ShapeId pick_shape(const BandedParams &p, int D, bool norm) {
   // few head rows without norm (Q, K and, for an FP8 cache, V), or Q converted to another
   // type: the light shape
-#ifdef ROPE_FP8_MID
-  if (!norm && p.band[0].kv8) return kMid;
-#endif
   if (!norm && (p.work_total <= 64 || p.band[0].q_conv)) return kLight;
-#ifdef ROPE_NORM_ALWAYS_MID
-  if (norm) return kMid;
-#endif
   return passes(p, D, kMidShape.cw) <= passes(p, D, kHeavyShape.cw) ? kMid : kHeavy;
 }
 
@@ -514,13 +511,15 @@ static rope_status_t launch_gemv_r(const GemvParams &p, cudaStream_t st) {
   return launch(gemv_norm_kernel<T, R, false>, grid, kGemvThreads, 0, st, p);
 }
 
-// rows per CTA: the fewest that keep the grid within one CTA per SM (at most 8)
+// rows per CTA: the fewest that keep the grid within four CTAs an SM (at most 8).  On the
+// latent-attention KV projection (W [576, 7168]) one row a CTA, 576 CTAs, ran 6.5 us a call
+// in a CUDA graph, against 6.7 with four rows (144 CTAs) and 7.0 with eight.
 template <typename T>
 static rope_status_t launch_gemv_t(const GemvParams &p, cudaStream_t st) {
   const int sms = sm_count() > 0 ? sm_count() : 1;
-  if (p.n <= sms) return launch_gemv_r<T, 1>(p, st);
-  if (p.n <= 2 * sms) return launch_gemv_r<T, 2>(p, st);
-  if (p.n <= 4 * sms) return launch_gemv_r<T, 4>(p, st);
+  if (p.n <= 4 * sms) return launch_gemv_r<T, 1>(p, st);
+  if (p.n <= 8 * sms) return launch_gemv_r<T, 2>(p, st);
+  if (p.n <= 16 * sms) return launch_gemv_r<T, 4>(p, st);
   return launch_gemv_r<T, 8>(p, st);
 }
 
