@@ -16,8 +16,9 @@
 //                      L = head_dim / (2 * vector) lanes; each lane owns two 16-byte vectors
 //                      of a row (for half-split RoPE the two halves of its rotation pairs),
 //                      normalises them (shuffle reduction over its group), rotates them and
-//                      writes them back in place, taking up to three of its rows at once so
-//                      that their dependency chains overlap (rows_step);
+//                      writes them back in place; with the norm, a first pass over up to
+//                      three of its rows reduces their sums of squares together, and a second
+//                      reads each row again to scale, rotate and write it (rows_step);
 //   warp 1, storer:    once the consumers are done with a token, bulk-copies the stage's Q
 //                      block to q_out and its K and V blocks to the cache page, waits until
 //                      the copies have read the stage, and hands the stage back.
@@ -70,11 +71,10 @@ struct BandDev {
   const float *k_scale, *v_scale;
 };
 
-// N float values written at shared address a as N E4M3 codes (nearest, ties to even,
-// saturating at +-448)
+// N float values as N E4M3 codes, code i in byte i % 4 of word i / 4 (nearest, ties to
+// even, saturating at +-448)
 template <int N>
-__device__ __forceinline__ void sts_e4m3(uint32_t a, const float (&x)[N]) {
-  uint32_t w[N / 4];
+__device__ __forceinline__ void e4m3_words(const float (&x)[N], uint32_t (&w)[N / 4]) {
 #pragma unroll
   for (int i = 0; i < N / 4; ++i) {
     const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * i], x[4 * i + 1]),
@@ -83,6 +83,11 @@ __device__ __forceinline__ void sts_e4m3(uint32_t a, const float (&x)[N]) {
                                                  __NV_SATFINITE, __NV_E4M3);
     w[i] = lo | (hi << 16);
   }
+}
+
+// The N / 4 code words of N values at shared address a
+template <int N>
+__device__ __forceinline__ void sts_words(uint32_t a, const uint32_t (&w)[N / 4]) {
   if constexpr (N == 8) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(a), "r"(w[0]), "r"(w[1]) : "memory");
   } else {
@@ -317,11 +322,10 @@ __device__ __forceinline__ void lds_freqs(const unsigned char *F, int fdt, int c
   }
 }
 
-// Head rows a consumer thread takes at once (overlapping their dependency chains), within
+// Head rows whose norm reductions a consumer thread overlaps (rows_step's first pass), within
 // the register budget of the shape: light CTAs run three to an SM, the others two.  Three
-// for the six-warp norm shape (the per-head norm ran 133, 128 and 117-119 us with one, two
-// and three), one elsewhere (the eight-warp shape has 96 registers, and a store without the
-// norm has short chains).
+// for the six-warp norm shape, one elsewhere (the eight-warp shape has 96 registers, and two
+// rows spilled there; a store without the norm has no reduction).
 #ifndef ROPE_CHUNK_ROWS_NORM
 #define ROPE_CHUNK_ROWS_NORM 3
 #endif
@@ -475,15 +479,18 @@ struct BandOut {
 
 // J head rows of a staged token, listed at it[0], it[stride], ...: optionally normalised
 // (per-head RMSNorm with the gamma rows at shared addresses gq / gk for Q / K rows), then
-// rotated with the token's table row F (INTER: the interleaved layout), written back in
-// place.  The J rows' dependency chains are interleaved.  EF: `fr` holds the table row
-// already; else it is read here, after the norm (so that it and the gammas are never live
-// together).  EXT: outputs as `bo` says.
-template <int J, typename T, int D, bool NORM, int L, bool INTER, bool EXT, bool EF>
+// rotated with the token's table row, held in `fr` (INTER: the interleaved layout), and
+// written back in place (EXT: outputs as `bo` says).  With the norm, a first pass reads the
+// J rows and reduces their sums of squares together, so that their shuffle and reciprocal
+// square-root latencies overlap while only one float a row stays live; the second pass reads
+// each row again (shared memory has the bandwidth to spare) and scales, rotates and writes
+// it.  Three rows held whole through the reduction spilled at 128 registers (per-head norm
+// 118.8 us, against 105 us for the two passes).
+template <int J, typename T, int D, bool NORM, int L, bool INTER, bool EXT>
 __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t *it, int stride,
                                           uint32_t st, uint32_t gq, uint32_t gk, float eps,
-                                          int mbc, const unsigned char *F,
-                                          LaneFreqs<Vec<T>::N, INTER> &fr, const BandOut &bo) {
+                                          int mbc, const LaneFreqs<Vec<T>::N, INTER> &fr,
+                                          const BandOut &bo) {
   using VT = Vec<T>;
   constexpr int N = VT::N, H2 = N / 2, EB = (int)sizeof(T);
   uint32_t row[J], g[J];
@@ -495,27 +502,24 @@ __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t
     isk[j] = ((w >> kItemKindShift) & 3) != 0;
     g[j] = isk[j] ? gk : gq;
   }
-  float2 xa[J][H2], xb[J][H2];
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    float t[N];
-    VT::widen(lds_v4(row[j] + cl.ca * EB), t);
-#pragma unroll
-    for (int k = 0; k < H2; ++k) xa[j][k] = make_float2(t[2 * k], t[2 * k + 1]);
-    VT::widen(lds_v4(row[j] + cl.cb * EB), t);
-#pragma unroll
-    for (int k = 0; k < H2; ++k) xb[j][k] = make_float2(t[2 * k], t[2 * k + 1]);
-  }
   float r[J];
   if constexpr (NORM) {
+    // first pass: each row's sum of squares, read straight from shared memory, so that only
+    // one float a row stays live across the reduction and the reciprocal square root
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-      float2 acc = __fmul2_rn(xa[j][0], xa[j][0]);
-      acc = __ffma2_rn(xb[j][0], xb[j][0], acc);
+      float ta[N], tb[N];
+      VT::widen(lds_v4(row[j] + cl.ca * EB), ta);
+      VT::widen(lds_v4(row[j] + cl.cb * EB), tb);
+      // pairs of the two vectors alternately, as two float32 lanes
+      float2 acc = __fmul2_rn(make_float2(ta[0], ta[1]), make_float2(ta[0], ta[1]));
+      acc = __ffma2_rn(make_float2(tb[0], tb[1]), make_float2(tb[0], tb[1]), acc);
 #pragma unroll
       for (int k = 1; k < H2; ++k) {
-        acc = __ffma2_rn(xa[j][k], xa[j][k], acc);
-        acc = __ffma2_rn(xb[j][k], xb[j][k], acc);
+        acc = __ffma2_rn(make_float2(ta[2 * k], ta[2 * k + 1]),
+                         make_float2(ta[2 * k], ta[2 * k + 1]), acc);
+        acc = __ffma2_rn(make_float2(tb[2 * k], tb[2 * k + 1]),
+                         make_float2(tb[2 * k], tb[2 * k + 1]), acc);
       }
       r[j] = acc.x + acc.y;
     }
@@ -523,10 +527,25 @@ __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t
     for (int msk = L / 2; msk > 0; msk >>= 1)
 #pragma unroll
       for (int j = 0; j < J; ++j) r[j] += __shfl_xor_sync(cl.gmask, r[j], msk);
-    float ga[N], gb[N];  // gamma + weight_offset of the lane's columns, read once per kind
 #pragma unroll
-    for (int j = 0; j < J; ++j) {
-      r[j] = rsqrtf(r[j] * (1.0f / D) + eps);
+    for (int j = 0; j < J; ++j) r[j] = rsqrtf(r[j] * (1.0f / D) + eps);
+  }
+  // row by row (the second pass with the norm): read the row, scale, rotate, write
+  float ga[N], gb[N];  // gamma + weight_offset of the lane's columns, read once per kind
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    float2 xa[H2], xb[H2];
+    {
+      float t[N];
+      VT::widen(lds_v4(row[j] + cl.ca * EB), t);
+#pragma unroll
+      for (int k = 0; k < H2; ++k) xa[k] = make_float2(t[2 * k], t[2 * k + 1]);
+      VT::widen(lds_v4(row[j] + cl.cb * EB), t);
+#pragma unroll
+      for (int k = 0; k < H2; ++k) xb[k] = make_float2(t[2 * k], t[2 * k + 1]);
+    }
+    float rj = 1.f;
+    if constexpr (NORM) {
       if (j == 0 || g[j] != g[j - 1]) {
         lds_f32<N>(g[j] + cl.ca * 4, cl.li, ga);
         lds_f32<N>(g[j] + cl.cb * 4, cl.li, gb);
@@ -534,41 +553,37 @@ __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t
       if (mbc) {  // x * gamma now; the scalar r after the rotation
 #pragma unroll
         for (int k = 0; k < H2; ++k) {
-          xa[j][k] = __fmul2_rn(xa[j][k], make_float2(ga[2 * k], ga[2 * k + 1]));
-          xb[j][k] = __fmul2_rn(xb[j][k], make_float2(gb[2 * k], gb[2 * k + 1]));
+          xa[k] = __fmul2_rn(xa[k], make_float2(ga[2 * k], ga[2 * k + 1]));
+          xb[k] = __fmul2_rn(xb[k], make_float2(gb[2 * k], gb[2 * k + 1]));
         }
+        rj = r[j];
       } else {  // the normalised value is rounded to the element type, then scaled
         const float2 rr = make_float2(r[j], r[j]);
 #pragma unroll
         for (int k = 0; k < H2; ++k) {
-          xa[j][k] = __fmul2_rn(round2<T>(__fmul2_rn(xa[j][k], rr)),
+          xa[k] = __fmul2_rn(round2<T>(__fmul2_rn(xa[k], rr)),
                                 make_float2(ga[2 * k], ga[2 * k + 1]));
-          xb[j][k] = __fmul2_rn(round2<T>(__fmul2_rn(xb[j][k], rr)),
+          xb[k] = __fmul2_rn(round2<T>(__fmul2_rn(xb[k], rr)),
                                 make_float2(gb[2 * k], gb[2 * k + 1]));
         }
-        r[j] = 1.f;
       }
     }
-    if constexpr (!EF) load_lane_freqs<N, INTER>(fr, cl, F);
-  }
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    rotate_lane<H2, INTER>(fr, cl, xa[j], xb[j]);
+    rotate_lane<H2, INTER>(fr, cl, xa, xb);
     if constexpr (NORM) {
-      const float2 rr = make_float2(r[j], r[j]);
+      const float2 rr = make_float2(rj, rj);
 #pragma unroll
       for (int k = 0; k < H2; ++k) {
-        xa[j][k] = __fmul2_rn(xa[j][k], rr);
-        xb[j][k] = __fmul2_rn(xb[j][k], rr);
+        xa[k] = __fmul2_rn(xa[k], rr);
+        xb[k] = __fmul2_rn(xb[k], rr);
       }
     }
     float ta[N], tb[N];
 #pragma unroll
     for (int k = 0; k < H2; ++k) {
-      ta[2 * k] = xa[j][k].x;
-      ta[2 * k + 1] = xa[j][k].y;
-      tb[2 * k] = xb[j][k].x;
-      tb[2 * k + 1] = xb[j][k].y;
+      ta[2 * k] = xa[k].x;
+      ta[2 * k + 1] = xa[k].y;
+      tb[2 * k] = xb[k].x;
+      tb[2 * k + 1] = xb[k].y;
     }
     if constexpr (EXT) {
       const int rb = (int)(row[j] - bo.blk) / (D * EB);  // the row's index in the band block
@@ -585,8 +600,20 @@ __device__ __forceinline__ void rows_step(const ConsumerLane &cl, const uint32_t
           tb[e] *= bo.kinv;
         }
         const uint32_t krow = bo.k8 + (uint32_t)((rb - bo.n_q) * D);
-        sts_e4m3<N>(krow + cl.ca, ta);
-        sts_e4m3<N>(krow + cl.cb, tb);
+        uint32_t wa[N / 4], wb[N / 4], w1[N / 4], w2[N / 4];
+        e4m3_words<N>(ta, wa);
+        e4m3_words<N>(tb, wb);
+        // the row groups of a warp sit one code row (128 bytes at head_dim 128) apart, on the
+        // same banks: odd groups store their b half first, so that each store instruction
+        // covers all 32 banks
+        const bool odd = (threadIdx.x / L) & 1;
+#pragma unroll
+        for (int e = 0; e < N / 4; ++e) {
+          w1[e] = odd ? wb[e] : wa[e];
+          w2[e] = odd ? wa[e] : wb[e];
+        }
+        sts_words<N>(krow + (odd ? cl.cb : cl.ca), w1);
+        sts_words<N>(krow + (odd ? cl.ca : cl.cb), w2);
         continue;
       }
     }
@@ -612,8 +639,10 @@ __device__ __forceinline__ void v_rows(const ConsumerLane &cl, const uint32_t *i
     float x[2][N];
     VT::widen(lds_v4(row + cl.ca * EB), x[0]);
     VT::widen(lds_v4(row + cl.cb * EB), x[1]);
+    const int odd = (threadIdx.x / (D / (2 * N))) & 1;  // b half first, as for the K codes
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h0 = 0; h0 < 2; ++h0) {
+      const int h = h0 ^ odd;
       const uint32_t a = vrow + (h ? cl.cb : cl.ca);
       const uint32_t w0 = bo.v_pow2 ? e4m3_scaled4(x[h][0], x[h][1], x[h][2], x[h][3], bo.vinv)
                                     : e4m3_exact4(x[h][0], x[h][1], x[h][2], x[h][3], bo.vinv,
@@ -630,30 +659,29 @@ __device__ __forceinline__ void v_rows(const ConsumerLane &cl, const uint32_t *i
   }
 }
 
-// A band's slots [lo, hi) of a consumer thread's head rows, JM at a time.  Without the norm,
-// or one row at a time, the table row is read once here, for every chunk.
+// A band's slots [lo, hi) of a consumer thread's head rows, JM at a time; the token's table
+// row is read once here, for every chunk.
 template <int JM, typename T, int D, bool NORM, int L, bool INTER, bool EXT>
 __device__ __forceinline__ void rows_band(const ConsumerLane &cl, const uint32_t *item, int stride,
                                           int lo, int hi, uint32_t st, uint32_t gq, uint32_t gk,
                                           float eps, int mbc, const unsigned char *F,
                                           const BandOut &bo) {
-  constexpr bool EF = !NORM || JM == 1;
   LaneFreqs<Vec<T>::N, INTER> fr;
-  if constexpr (EF) load_lane_freqs<Vec<T>::N, INTER>(fr, cl, F);
+  load_lane_freqs<Vec<T>::N, INTER>(fr, cl, F);
   int u = lo;
 #pragma unroll 1
   for (; u + JM <= hi; u += JM)
-    rows_step<JM, T, D, NORM, L, INTER, EXT, EF>(cl, item + u * stride, stride, st, gq, gk, eps,
-                                                 mbc, F, fr, bo);
+    rows_step<JM, T, D, NORM, L, INTER, EXT>(cl, item + u * stride, stride, st, gq, gk, eps,
+                                             mbc, fr, bo);
   if constexpr (JM >= 3) {
     if (hi - u == 2)
-      rows_step<2, T, D, NORM, L, INTER, EXT, EF>(cl, item + u * stride, stride, st, gq, gk, eps,
-                                                  mbc, F, fr, bo);
+      rows_step<2, T, D, NORM, L, INTER, EXT>(cl, item + u * stride, stride, st, gq, gk, eps,
+                                              mbc, fr, bo);
   }
   if constexpr (JM >= 2) {
     if (hi - u == 1)
-      rows_step<1, T, D, NORM, L, INTER, EXT, EF>(cl, item + u * stride, stride, st, gq, gk, eps,
-                                                  mbc, F, fr, bo);
+      rows_step<1, T, D, NORM, L, INTER, EXT>(cl, item + u * stride, stride, st, gq, gk, eps,
+                                              mbc, fr, bo);
   }
 }
 
