@@ -80,9 +80,27 @@ def parse_args():
 
 # ------------------------------------------------------------------ small utilities --
 
-def kernel_source_hash() -> str:
+# the kernel files each entry point's kernel is built from, beyond the host code and the
+# shared device headers (radd's kernel includes the banded one's header)
+KERNEL_FILES = {"rope_split_store_paged_ragged": ("banded.cuh",),
+                "fused_qk_rmsnorm_rope_paged": ("banded.cuh",),
+                "fused_dual_qk_rmsnorm_rope_paged": ("banded.cuh",),
+                "kv_cache_radd": ("banded.cuh", "radd.cuh"),
+                "qk_rope_bshd_continuous": ("bshd.cuh",),
+                "matmul_fused_partial_rmsnorm": ("gemv_norm.cuh",)}
+SHARED_SOURCES = ("rope_store.cu", "common.cuh", "pipeline.cuh", "device_utils.cuh")
+
+
+def kernel_source_hash(workload=None) -> str:
+    """sha256 (first 16 hex digits) of the sources the workload's kernel is built from (the
+    host code, the shared device headers and its kernel's files), or of every kernel source."""
+    if workload is None:
+        files = KERNEL_SOURCES
+    else:
+        files = ["rope_paged_kv_b200/csrc/" + f
+                 for f in SHARED_SOURCES + KERNEL_FILES[WORKLOADS[workload]]]
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -112,7 +130,7 @@ def profiled_traffic(workload):
     text = open(p).read()
     m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(workload):
         return None
     return int(m_bytes.group(1))
 
