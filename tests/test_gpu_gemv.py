@@ -89,6 +89,39 @@ def test_two_calls_in_a_row_share_a_workspace(rs):
         H.assert_close_bf16(H.bits(d["unnormed_output"]), r.unnormed, "unnormed")
 
 
+def test_chained_calls_under_early_overlap(rs):
+    """Launch-overlap mode 2 (programmatic dependent launch): the second call's x is the
+    first call's output, queued without a sync in between, so a read of x before the wait
+    for the preceding kernel would see the sentinel bits."""
+    import dataclasses
+    w1 = W.gemv_norm(74, n=1024, k=512, n_normed=0)
+    w2 = W.gemv_norm(75, n=576, k=1024, n_normed=512)
+    d1 = {f: getattr(w1, f).to(DEV) for f in ("x", "weight", "gamma", "normed_output",
+                                              "unnormed_output")}
+    d2 = {f: getattr(w2, f).to(DEV) for f in ("weight", "gamma", "normed_output",
+                                              "unnormed_output")}
+    ws1, ws2 = rs.gemv_workspace(0, DEV), rs.gemv_workspace(512, DEV)
+    before = rs.get_launch_overlap()
+    rs.set_launch_overlap(2)
+    try:
+        for _ in range(3):  # the later rounds run behind the earlier ones' kernels
+            rs.matmul_fused_partial_rmsnorm(d1["x"], d1["weight"], d1["gamma"], w1.epsilon, 0.0,
+                                            d1["normed_output"], d1["unnormed_output"], ws1)
+            rs.matmul_fused_partial_rmsnorm(d1["unnormed_output"], d2["weight"], d2["gamma"],
+                                            w2.epsilon, 0.0, d2["normed_output"],
+                                            d2["unnormed_output"], ws2)
+        torch.cuda.synchronize()
+    finally:
+        rs.set_launch_overlap(before)
+    r1 = H.oracle_gemv(w1)
+    H.assert_close_bf16(H.bits(d1["unnormed_output"]), r1.unnormed, "first call")
+    y1 = d1["unnormed_output"].cpu()
+    r2 = H.oracle_gemv(dataclasses.replace(w2, x=y1))
+    H.assert_close_bf16(H.bits(d2["normed_output"]), r2.normed, "normed")
+    H.assert_close_bf16(H.bits(d2["unnormed_output"]), r2.unnormed, "unnormed")
+    assert int(ws2[0].item()) == 0
+
+
 def test_argument_errors(rs):
     lib = rs.raw_library()
     x = torch.zeros(64, dtype=torch.bfloat16, device=DEV)
