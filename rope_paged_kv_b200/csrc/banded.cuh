@@ -666,6 +666,7 @@ __device__ __forceinline__ void rows_band(const ConsumerLane &cl, const uint32_t
                                           int lo, int hi, uint32_t st, uint32_t gq, uint32_t gk,
                                           float eps, int mbc, const unsigned char *F,
                                           const BandOut &bo) {
+  static_assert(JM >= 1 && JM <= 3, "the tail below takes at most two rows after the chunks");
   LaneFreqs<Vec<T>::N, INTER> fr;
   load_lane_freqs<Vec<T>::N, INTER>(fr, cl, F);
   int u = lo;
