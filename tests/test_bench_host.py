@@ -164,3 +164,34 @@ def test_batch_prefix_takes_the_first_sequences_of_the_batch():
     assert w.total_tokens == 5000 and w.lengths[:-1] == full.lengths[:k - 1]
     assert w.lengths[-1] <= full.lengths[k - 1]
     assert w.cache_lengths_of(w.main_cache) == full.cache_lengths_of(full.main_cache)[:k]
+
+
+def test_source_hash_of_each_workload_covers_its_kernel_files():
+    """A summary's hash covers the host code, the shared device headers and its kernel's
+    files: workloads of one kernel share it, and editing one kernel's file leaves the other
+    kernels' hashes as they were (checked on a copy of the sources)."""
+    import shutil
+    import tempfile
+    import bench
+    by_kernel = {}
+    for w in bench.WORKLOADS:
+        h = bench.kernel_source_hash(w)
+        assert len(h) == 16 and int(h, 16) >= 0
+        by_kernel.setdefault(bench.KERNEL_FILES[bench.WORKLOADS[w]], set()).add(h)
+    assert all(len(v) == 1 for v in by_kernel.values())
+    assert len({next(iter(v)) for v in by_kernel.values()}) == len(by_kernel)
+    with tempfile.TemporaryDirectory() as d:
+        shutil.copytree(os.path.join(bench.ROOT, "rope_paged_kv_b200", "csrc"),
+                        os.path.join(d, "rope_paged_kv_b200", "csrc"))
+        root = bench.ROOT
+        try:
+            bench.ROOT = d
+            before = {w: bench.kernel_source_hash(w) for w in bench.WORKLOADS}
+            with open(os.path.join(d, "rope_paged_kv_b200", "csrc", "gemv_norm.cuh"), "a") as f:
+                f.write("\n")
+            after = {w: bench.kernel_source_hash(w) for w in bench.WORKLOADS}
+        finally:
+            bench.ROOT = root
+    changed = {w for w in before if before[w] != after[w]}
+    assert changed == {w for w in bench.WORKLOADS
+                       if bench.WORKLOADS[w] == "matmul_fused_partial_rmsnorm"}
