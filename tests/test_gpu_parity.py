@@ -251,6 +251,19 @@ def test_ragged_edge_cases(G, name, norm):
     check_ragged(G, w, G.run_ragged(w))
 
 
+@pytest.mark.parametrize("n_q,n_kv,mbc", [(32, 8, True), (40, 8, False), (60, 6, True),
+                                          (64, 8, True)])
+def test_norm_rows_a_thread(G, n_q, n_kv, mbc):
+    """The norm's row steps take a thread's rows three at a time, then a tail of one or two.
+    In the six-warp shape (24 row groups) Q + K rows of 40 give threads two and one rows, 48
+    two, 66 three and two, 72 three: every step size, with either order of cast and gamma."""
+    w = W.ragged_store(1300 + n_q + n_kv, lengths=[70, 1, 33], cache_lengths=[0, 11, 90],
+                       n_q_heads=n_q, n_kv_heads=n_kv, head_dim=128, page_size=32, rope_dim=128,
+                       theta=1e4, interleaved=False, max_seq_len=256, norm=True, epsilon=1e-6,
+                       x_std=2.0, weight_offset=0.25)
+    check_ragged(G, w, G.run_ragged(w, multiply_before_cast=mbc), multiply_before_cast=mbc)
+
+
 def test_norm_weight_offset_one(G):
     w = W.ragged_store(1201, lengths=[40, 25], cache_lengths=[0, 9], n_q_heads=8, n_kv_heads=2,
                        head_dim=128, page_size=16, rope_dim=128, theta=1e4, interleaved=False,
